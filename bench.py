@@ -1,0 +1,356 @@
+"""Benchmark of the SharQ linear layer on B200: one JSON line on rank 0.
+
+A step is one pass of the per-token hot path on one batch: the fused preparation
+operator (RMSNorm + 2:4-pair mask + NVFP4 backbone + residual + NVFP4 residual) and
+the SharQ linear (sparse FP4 MMA + dense FP4 MMA into one accumulator + epilogue),
+on the Llama-3.1-8B QKV projection at prefill (X [2048, 4096] bf16, W [6144, 4096]).
+The weight is packed once before timing (an offline step).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sharq|reference]
+
+--impl reference times the CPU oracle (oracle/, NumPy) on bounded row samples of the
+same workload. Multi-GPU runs (torchrun, one rank per GPU) are replicas: token rows are
+independent, every rank processes its own batch with no data-path collective
+("scaling": "weak"); NCCL only carries the barrier and the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "SharQ linear tokens/s & eff. FP4 TFLOPS (Llama-8B shapes); prep HBM GB/s"
+L2_BYTES = 126 * 2 ** 20
+# algorithmic bytes of the preparation operator per activation element, NVFP4, 2:4 pairs:
+# 2 (bf16 x) + 1/4 (backbone codes) + 1/16 (metadata) + 1/32 (backbone scales)
+# + 1/2 (residual codes) + 1/16 (residual scales); + 4 bytes per row (s_x), gamma once.
+PREP_BYTES_PER_ELEM = 2 + 0.25 + 1 / 16 + 1 / 32 + 0.5 + 1 / 16
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.seek(0)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.file.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.file.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def to_dev(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+# --------------------------------------------------------------------------- CPU oracle arm
+def oracle_throughput(lin, rows_per_step: int, steps: int, warmup: int):
+    """Tokens/s of the CPU oracle (prep + float64 GEMM) on row samples; weight packed outside."""
+    from oracle import sharq as O
+    wp = O.pack_weight(wl.bf16_bits_to_f32(lin.w), O.NVFP4)
+    g = wl.bf16_bits_to_f32(lin.gamma)
+    T = lin.x.shape[0]
+    total, rows_done = 0.0, 0
+    for i in range(warmup + steps):
+        r0 = (i * rows_per_step) % T
+        x = wl.bf16_bits_to_f32(lin.x[r0:r0 + rows_per_step])
+        t0 = time.perf_counter()
+        p = O.prepare(x, g, lin.eps, 2, 4, 2, O.NVFP4)
+        O.linear(p, wp)
+        dt = time.perf_counter() - t0
+        if i >= warmup:
+            total += dt
+            rows_done += x.shape[0]
+    return rows_done / total, total, rows_done
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    lin = wl.llama_qkv(T=2048)
+    T, K, N = lin.shape
+    rows = 128
+    tps, secs, done = oracle_throughput(lin, rows, args.steps, min(args.warmup, 1))
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded outlier-channel activations, N(0,0.02) weight)",
+        "config": {"workload": f"llama31_8b_qkv_prefill T={T} K={K} N={N} nvfp4 2:4-pairs fused-rmsnorm",
+                   "rows_per_step": rows},
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} token rows per step x {args.steps} steps (prep + float64 GEMM vs all "
+                                   f"{N} outputs); weight packed once outside timing"},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- SharQ arm
+def run_sharq(args, rank, world, local):
+    import fp4_activation_sparse_b200 as S
+    hbm_peak, bf16_peak, bf16_sust, peak_src = load_peaks()
+    fp4_dense_peak = bf16_peak * 4.0  # nominal FP4:BF16 dense ratio 9 : 2.25 applied to the measured bf16 peak
+
+    lin = wl.llama_qkv(T=2048, seed=1 + rank)
+    T, K, N = lin.shape
+    # input sets rotated so each step touches data last used > L2 bytes earlier
+    w_dev = to_dev(lin.w)
+    footprint = T * K * 2 + T * K * 0.95 + N * K * 0.6 + T * N * 2
+    nsets = max(3, int(np.ceil(3 * L2_BYTES / footprint)))
+    xs = [to_dev(lin.x) for _ in range(nsets)]
+    gamma = to_dev(lin.gamma)
+    wps = [S.sharq_pack_weight(w_dev, "nvfp4") for _ in range(nsets)]
+    preps = [S.alloc_prep(T, K, 2, 4, 2, "nvfp4") for _ in range(nsets)]
+    ys = [torch.empty(T, N, dtype=torch.bfloat16, device="cuda") for _ in range(nsets)]
+    del w_dev
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        s = i % nsets
+        S.sharq_prepare(xs[s], gamma, lin.eps, 2, 4, 2, "nvfp4", out=preps[s], stream=stream)
+        S.sharq_linear(preps[s], wps[s], y=ys[s], stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert S.sharq_device_status() == S.SHARQ_OK
+
+    # ---- device-timed whole steps
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
+    clocks = clk.summary()
+
+    # ---- per-kernel times (events around each launch on the launching stream)
+    def per_kernel(n):
+        tp, tl = [], []
+        for i in range(n):
+            s = i % nsets
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record(stream)
+            S.sharq_prepare(xs[s], gamma, lin.eps, 2, 4, 2, "nvfp4", out=preps[s], stream=stream)
+            e[1].record(stream)
+            S.sharq_linear(preps[s], wps[s], y=ys[s], stream=stream)
+            e[2].record(stream)
+            e[2].synchronize()
+            tp.append(e[0].elapsed_time(e[1]))
+            tl.append(e[1].elapsed_time(e[2]))
+        return statistics.median(tp), statistics.median(tl)
+
+    t_prep_ms, t_lin_ms = per_kernel(max(args.steps, 10))
+
+    # ---- baselines on the same shapes: torch bf16 matmul and the library's dense NVFP4 pipeline
+    q = S.sharq_quantize_dense(xs[0], gamma, lin.eps, "nvfp4")
+    yd = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
+    w_bf16 = to_dev(lin.w)
+
+    def timeit(f, n=20):
+        for _ in range(3):
+            f()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            f()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b) / n
+
+    t_bf16 = timeit(lambda: torch.matmul(xs[0], w_bf16.t()))
+    t_dq = timeit(lambda: S.sharq_quantize_dense(xs[0], gamma, lin.eps, "nvfp4", out=q, stream=stream))
+    t_dl = timeit(lambda: S.sharq_linear_dense(q, wps[0], y=yd, stream=stream))
+    del w_bf16
+
+    # ---- end to end through the public API with host buffers (H2D x, D2H y inside the timing)
+    x_host = torch.from_numpy(np.ascontiguousarray(lin.x).view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_host = torch.empty(T, N, dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step(i):
+        s = i % nsets
+        xs[s].copy_(x_host, non_blocking=True)
+        S.sharq_prepare(xs[s], gamma, lin.eps, 2, 4, 2, "nvfp4", out=preps[s], stream=stream)
+        S.sharq_linear(preps[s], wps[s], y=ys[s], stream=stream)
+        y_host.copy_(ys[s], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_e2e = max_over_ranks(a.elapsed_time(b), world)
+    status = S.sharq_device_status()
+
+    if rank != 0:
+        return
+    tokens = T * args.steps * world
+    value = tokens / (ms_total / 1e3)
+    eff_tflops = 2.0 * T * N * K * args.steps * world / (ms_total / 1e3) / 1e12
+    prep_bytes = T * K * PREP_BYTES_PER_ELEM + T * 4 + K * 2
+    prep_gbs = prep_bytes / (t_prep_ms / 1e3) / 1e9
+    gemm_work = 3.0 * T * N * K  # dense-equivalent tensor work: sparse path T*N*K, dense path 2*T*N*K
+    gemm_tflops = gemm_work / (t_lin_ms / 1e3) / 1e12
+    rf_prep = {"bound": "hbm", "achieved": prep_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": prep_gbs / hbm_peak,
+               "traffic": None, "kernel": "sharq_prep", "peak_source": peak_src}
+    rf_gemm = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_dense_peak, "unit": "TFLOP/s",
+               "frac": gemm_tflops / fp4_dense_peak, "traffic": None, "kernel": "sharq_gemm",
+               "peak_source": f"{peak_src} bf16 x 4 (nominal dense FP4:BF16)"}
+    dominant = rf_gemm if t_lin_ms >= t_prep_ms else rf_prep
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp4 (e2m1, e4m3 scales), fp32 accumulate",
+        "data": "synthetic (seeded outlier-channel activations, N(0,0.02) weight)",
+        "config": {"workload": f"llama31_8b_qkv_prefill T={T} K={K} N={N} nvfp4 2:4-pairs fused-rmsnorm",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single",
+                   "l2": f"{nsets} rotating input sets ({nsets * footprint / 2**20:.0f} MiB > L2)"},
+        "eff_fp4_tflops": eff_tflops, "prep_gbs": prep_gbs,
+        "t_prep_us": t_prep_ms * 1e3, "t_linear_us": t_lin_ms * 1e3,
+        "roofline": dominant, "roofline_prep": rf_prep, "roofline_gemm": rf_gemm,
+        "baselines": {"torch_bf16_matmul_us": t_bf16 * 1e3,
+                      "dense_nvfp4_pipeline_us": (t_dq + t_dl) * 1e3,
+                      "dense_nvfp4_quantize_us": t_dq * 1e3, "dense_nvfp4_gemm_us": t_dl * 1e3},
+        "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * K * 2,
+                "d2h_bytes_per_step": T * N * 2},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        tps, secs, done = oracle_throughput(lin, 128, 8, 1)
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"8 steps x 128 token rows (prep + float64 GEMM vs all {N} outputs), "
+                                          f"{secs:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["sharq", "reference"], default="sharq")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_sharq(args, rank, world, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,259 @@
+"""Python binding of libsharq: SharQ's online sparse-dense FP4 linear layer on B200.
+
+Argument marshalling only (ctypes). Every computation runs in the library's CUDA
+kernels; torch supplies device memory and streams. There is no CPU fallback: if
+``libsharq.so`` is missing, importing this package raises.
+
+The three calls of the method ("SharQ: Bridging Activation Sparsity and FP4
+Quantization for LLM Inference", Abstract):
+  sharq_pack_weight  - one FP4 weight payload with sparse-path and dense-path scale views
+  sharq_prepare      - the fused preparation operator (RMSNorm, N:M mask, FP4 backbone,
+                       residual against the quantized backbone, dense FP4 residual)
+  sharq_linear       - sparse FP4 GEMM + dense FP4 GEMM into one output
+and the library's dense FP4 baseline (the README's "NVFP4" mode):
+  sharq_quantize_dense, sharq_linear_dense.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsharq.so")
+
+SHARQ_NVFP4, SHARQ_MXFP4 = 0, 1
+SHARQ_OUT_BF16, SHARQ_OUT_F32 = 0, 1
+SHARQ_OK, SHARQ_ERR_INVALID_ARG, SHARQ_ERR_UNSUPPORTED, SHARQ_ERR_CUDA, SHARQ_ERR_TIMEOUT = range(5)
+FMT = {"nvfp4": SHARQ_NVFP4, "mxfp4": SHARQ_MXFP4}
+UNIT_ELEMENT, UNIT_PAIR = 1, 2
+
+
+class SharqError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"sharq status {status}: {message}")
+        self.status = status
+
+
+class _Prep(ctypes.Structure):
+    _fields_ = [("sparse_codes", ctypes.c_void_p), ("sparse_meta", ctypes.c_void_p),
+                ("sparse_scales", ctypes.c_void_p), ("resid_codes", ctypes.c_void_p),
+                ("resid_scales", ctypes.c_void_p), ("row_scale", ctypes.c_void_p),
+                ("tokens", ctypes.c_int), ("k", ctypes.c_int), ("nm_n", ctypes.c_int),
+                ("nm_m", ctypes.c_int), ("unit", ctypes.c_int), ("fmt", ctypes.c_int)]
+
+
+class _WPack(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales_sparse", ctypes.c_void_p),
+                ("scales_dense", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
+                ("n_out", ctypes.c_int), ("k", ctypes.c_int), ("fmt", ctypes.c_int)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m fp4_activation_sparse_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "sharq_prep_buffer_sizes": (S, [I, I, I, I, I, I, ctypes.POINTER(S)]),
+        "sharq_wpack_buffer_sizes": (S, [I, I, I, ctypes.POINTER(S)]),
+        "sharq_pack_weight": (I, [P, I, I, I, ctypes.POINTER(_WPack), P]),
+        "sharq_prepare": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P]),
+        "sharq_linear": (I, [ctypes.POINTER(_Prep), ctypes.POINTER(_WPack), P, I, P]),
+        "sharq_quantize_dense": (I, [P, I, I, P, F, I, P, P, P, P]),
+        "sharq_linear_dense": (I, [P, P, P, I, I, ctypes.POINTER(_WPack), P, I, P]),
+        "sharq_device_status": (I, [P]),
+        "sharq_set_wait_limit": (None, [ctypes.c_longlong]),
+        "sharq_last_error": (ctypes.c_char_p, []),
+        "sharq_version": (I, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    return lib
+
+
+lib = _load()
+
+
+def last_error() -> str:
+    return lib.sharq_last_error().decode()
+
+
+def _check(status: int):
+    if status != SHARQ_OK:
+        raise SharqError(status, last_error())
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _fmt(fmt) -> int:
+    return FMT[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+# ------------------------------------------------------------------ buffer holders
+@dataclass
+class Prep:
+    """A prepared activation: the six device buffers of ``sharq_prep`` and the C struct."""
+    sparse_codes: torch.Tensor
+    sparse_meta: torch.Tensor
+    sparse_scales: torch.Tensor
+    resid_codes: torch.Tensor
+    resid_scales: torch.Tensor
+    row_scale: torch.Tensor
+    tokens: int
+    k: int
+    nm_n: int
+    nm_m: int
+    unit: int
+    fmt: int
+    c: _Prep = field(default=None, repr=False)
+
+    def struct(self) -> _Prep:
+        if self.c is None:
+            self.c = _Prep(self.sparse_codes.data_ptr(), self.sparse_meta.data_ptr(), self.sparse_scales.data_ptr(),
+                           self.resid_codes.data_ptr(), self.resid_scales.data_ptr(), self.row_scale.data_ptr(),
+                           self.tokens, self.k, self.nm_n, self.nm_m, self.unit, self.fmt)
+        return self.c
+
+
+@dataclass
+class WPack:
+    """A packed weight: codes, the two scale views and the tensor scale."""
+    codes: torch.Tensor
+    scales_sparse: torch.Tensor
+    scales_dense: torch.Tensor
+    tensor_scale: torch.Tensor
+    n_out: int
+    k: int
+    fmt: int
+    c: _WPack = field(default=None, repr=False)
+
+    def struct(self) -> _WPack:
+        if self.c is None:
+            self.c = _WPack(self.codes.data_ptr(), self.scales_sparse.data_ptr(), self.scales_dense.data_ptr(),
+                            self.tensor_scale.data_ptr(), self.n_out, self.k, self.fmt)
+        return self.c
+
+
+def sharq_prep_buffer_sizes(tokens: int, k: int, nm_n: int, nm_m: int, unit: int, fmt) -> list[int]:
+    sizes = (ctypes.c_size_t * 6)()
+    if lib.sharq_prep_buffer_sizes(tokens, k, nm_n, nm_m, unit, _fmt(fmt), sizes) == 0:
+        raise SharqError(SHARQ_ERR_INVALID_ARG, last_error())
+    return list(sizes)
+
+
+def sharq_wpack_buffer_sizes(n_out: int, k: int, fmt) -> list[int]:
+    sizes = (ctypes.c_size_t * 4)()
+    if lib.sharq_wpack_buffer_sizes(n_out, k, _fmt(fmt), sizes) == 0:
+        raise SharqError(SHARQ_ERR_INVALID_ARG, last_error())
+    return list(sizes)
+
+
+def _bytes(n: int, device) -> torch.Tensor:
+    # 16-byte aligned (torch's caching allocator aligns to 512 bytes)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def alloc_prep(tokens: int, k: int, nm_n: int = 2, nm_m: int = 4, unit: int = UNIT_PAIR, fmt="nvfp4",
+               device="cuda") -> Prep:
+    s = sharq_prep_buffer_sizes(tokens, k, nm_n, nm_m, unit, fmt)
+    return Prep(_bytes(s[0], device), _bytes(s[1], device), _bytes(s[2], device), _bytes(s[3], device),
+                _bytes(s[4], device), torch.empty(tokens, dtype=torch.float32, device=device),
+                tokens, k, nm_n, nm_m, unit, _fmt(fmt))
+
+
+def alloc_wpack(n_out: int, k: int, fmt="nvfp4", device="cuda") -> WPack:
+    s = sharq_wpack_buffer_sizes(n_out, k, fmt)
+    return WPack(_bytes(s[0], device), _bytes(s[1], device), _bytes(s[2], device),
+                 torch.empty(4, dtype=torch.float32, device=device), n_out, k, _fmt(fmt))
+
+
+# ------------------------------------------------------------------ the calls
+def sharq_pack_weight(w: torch.Tensor, fmt="nvfp4", out: WPack | None = None, stream=None) -> WPack:
+    """Pack a bf16 weight [n_out, k] (device) into one FP4 payload with two scale views."""
+    assert w.dtype == torch.bfloat16 and w.is_cuda and w.is_contiguous()
+    n_out, k = w.shape
+    out = out or alloc_wpack(n_out, k, fmt, w.device)
+    st = out.struct()
+    _check(lib.sharq_pack_weight(_ptr(w), n_out, k, _fmt(fmt), ctypes.byref(st), _stream(stream)))
+    return out
+
+
+def sharq_prepare(x: torch.Tensor, gamma: torch.Tensor | None = None, eps: float = 1e-6, nm_n: int = 2,
+                  nm_m: int = 4, unit: int = UNIT_PAIR, fmt="nvfp4", out: Prep | None = None, stream=None) -> Prep:
+    """The fused preparation operator on bf16 activations [tokens, k] (device)."""
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous()
+    tokens, k = x.shape
+    if gamma is not None:
+        assert gamma.dtype == torch.bfloat16 and gamma.is_cuda and gamma.numel() == k
+    out = out or alloc_prep(tokens, k, nm_n, nm_m, unit, fmt, x.device)
+    st = out.struct()
+    _check(lib.sharq_prepare(_ptr(x), tokens, k, _ptr(gamma), ctypes.c_float(eps), nm_n, nm_m, unit, _fmt(fmt),
+                             ctypes.byref(st), _stream(stream)))
+    return out
+
+
+def sharq_linear(prep: Prep, w: WPack, y: torch.Tensor | None = None, out_dtype=torch.bfloat16,
+                 stream=None) -> torch.Tensor:
+    """Y [tokens, n_out] = sparse FP4 GEMM (backbone) + dense FP4 GEMM (residual), one output."""
+    if y is None:
+        y = torch.empty(prep.tokens, w.n_out, dtype=out_dtype, device=prep.resid_codes.device)
+    code = SHARQ_OUT_F32 if y.dtype == torch.float32 else SHARQ_OUT_BF16
+    _check(lib.sharq_linear(ctypes.byref(prep.struct()), ctypes.byref(w.struct()), _ptr(y), code, _stream(stream)))
+    return y
+
+
+@dataclass
+class DenseQ:
+    codes: torch.Tensor
+    scales: torch.Tensor
+    row_scale: torch.Tensor
+    tokens: int
+    k: int
+    fmt: int
+
+
+def sharq_quantize_dense(x: torch.Tensor, gamma: torch.Tensor | None = None, eps: float = 1e-6, fmt="nvfp4",
+                         out: DenseQ | None = None, stream=None) -> DenseQ:
+    """The dense FP4 baseline quantizer (optional RMSNorm + block quantization of every element)."""
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous()
+    tokens, k = x.shape
+    if out is None:
+        s = sharq_prep_buffer_sizes(tokens, k, 2, 4, UNIT_PAIR, fmt)
+        out = DenseQ(_bytes(s[3], x.device), _bytes(s[4], x.device),
+                     torch.empty(tokens, dtype=torch.float32, device=x.device), tokens, k, _fmt(fmt))
+    _check(lib.sharq_quantize_dense(_ptr(x), tokens, k, _ptr(gamma), ctypes.c_float(eps), _fmt(fmt),
+                                    _ptr(out.codes), _ptr(out.scales), _ptr(out.row_scale), _stream(stream)))
+    return out
+
+
+def sharq_linear_dense(q: DenseQ, w: WPack, y: torch.Tensor | None = None, out_dtype=torch.bfloat16,
+                       stream=None) -> torch.Tensor:
+    """The dense FP4 baseline GEMM against the weight's dense-path scale view."""
+    if y is None:
+        y = torch.empty(q.tokens, w.n_out, dtype=out_dtype, device=q.codes.device)
+    code = SHARQ_OUT_F32 if y.dtype == torch.float32 else SHARQ_OUT_BF16
+    _check(lib.sharq_linear_dense(_ptr(q.codes), _ptr(q.scales), _ptr(q.row_scale), q.tokens, q.k,
+                                  ctypes.byref(w.struct()), _ptr(y), code, _stream(stream)))
+    return y
+
+
+def sharq_device_status(stream=None) -> int:
+    """Synchronize the stream; return (and clear) the status of the bounded device waits."""
+    return lib.sharq_device_status(_stream(stream))
+
+
+def sharq_set_wait_limit(nanoseconds: int) -> None:
+    """Test hook: time limit of the GEMM's bounded waits (0 restores the default of 4 s)."""
+    lib.sharq_set_wait_limit(int(nanoseconds))

@@ -1,0 +1,54 @@
+"""Build libsharq.so (all SharQ CUDA kernels + the C ABI) in-tree for sm_100a.
+
+Usage: python -m fp4_activation_sparse_b200.build [--verbose]
+nvcc cross-compiles without a GPU; the shared object lands next to this file.
+"""
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+CSRC = os.path.join(HERE, "csrc")
+LIB = os.path.join(HERE, "libsharq.so")
+SOURCES = ["sharq_api.cu", "sharq_prep.cu", "sharq_pack.cu", "sharq_gemm.cu"]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found")
+
+
+def build(verbose: bool = False, extra: list[str] | None = None) -> str:
+    srcs = [os.path.join(CSRC, s) for s in SOURCES]
+    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+           "--expt-relaxed-constexpr", "-I", os.path.join(HERE, "..", "include"), "-o", LIB + ".tmp", *srcs,
+           "-lcudart"]
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+    if extra:
+        cmd[1:1] = extra
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
+    if verbose:
+        sys.stderr.write(res.stdout + res.stderr)
+    os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIB):
+        return False
+    t = os.path.getmtime(LIB)
+    deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(HERE, "..", "include", "sharq.h")]
+    return all(os.path.getmtime(d) <= t for d in deps)
+
+
+if __name__ == "__main__":
+    print(build(verbose="--verbose" in sys.argv))

@@ -1,0 +1,524 @@
+// SharQ linear layer GEMM (K3): structured-sparse + dense block-scaled FP4 MMAs into one
+// tensor-memory accumulator, one epilogue.
+//
+// "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM Inference",
+// Abstract: "A sparse FP4 GEMM processes the backbone while a dense FP4 GEMM
+// compensates for both mask-induced activation loss and sparse-path quantization
+// error. The two paths share a single FP4 weight payload with path-specific scale
+// views." The README ("Benchmarks") enables "epilogue fusion" on this path.
+//
+// sm_100a design (one CTA per SM, persistent over 128 x 256 output tiles):
+//   warp 0       TMA producer: per K-tile of 256 it loads the residual codes (SW128),
+//                the compressed backbone codes (SW64), the weight codes (SW128), the
+//                backbone metadata and the four scale tiles (1-D bulk copies of
+//                pre-tiled 128x4 atoms). Each weight tile is loaded once and feeds
+//                both MMAs.
+//   warp 1       TMEM owner and MMA issuer: tcgen05.cp moves scales and metadata to
+//                tensor memory, then two tcgen05.mma.sp (K=128 logical, pairwise 4:8)
+//                and four dense tcgen05.mma (K=64) accumulate into one 128x256 fp32
+//                accumulator. Both paths carry the same per-row scale s_x, so one
+//                accumulator holds their sum.
+//   warps 2..5   epilogue: tcgen05.ld, y = acc * s_x[row] * s_w, bf16/fp32 stores.
+// Every mbarrier wait is bounded by a time limit; on expiry the CTA records a status
+// word, stops issuing, waits (bounded) for its own copies and MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "sharq_common.cuh"
+#include "sharq_internal.h"
+
+namespace sharq {
+
+__device__ uint32_t g_device_status = 0;  // bit 0: a bounded wait gave up
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 256;  // BK in logical K elements
+constexpr int kStages = 3;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCols = 256;
+constexpr uint32_t kScaleBufCols = 80;  // per K-tile parity: meta 4, SFA_sp 8, SFA_res 16, SFB_sp 16, SFB_res 32
+// Drains (own copies and MMAs in flight before exit) always get the full bound, also when a
+// test lowers the limit of the ordinary waits.
+constexpr uint64_t kDrainLimitNs = 4000000000ull;
+
+// shared-memory stage layout (bytes)
+constexpr int OFF_ARES = 0;       // 128 rows x 128 B, SW128
+constexpr int OFF_B = 16384;      // 256 rows x 128 B, SW128
+constexpr int OFF_ASP = 49152;    // 128 rows x 64 B, SW64
+constexpr int OFF_META = 57344;   // 128 rows x 16 B
+constexpr int OFF_SFA_RES = 59392;
+constexpr int OFF_SFA_SP = 61440;
+constexpr int OFF_SFB_RES = 62464;  // n-block 0 at +0, n-block 1 at +2048
+constexpr int OFF_SFB_SP = 66560;   // n-block 0 at +0, n-block 1 at +1024
+constexpr int kStageBytes = 68608;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align slack*/ + 256 /*barriers*/;
+
+struct __align__(64) TmaMaps {
+  CUtensorMap a_res, a_sp, b;
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait: gives up after `limit_ns` (or when another role of the CTA already
+// gave up) and records the failure in the device status word.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                          volatile uint32_t *abort_flag) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if (i == 1 || (i & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > limit_ns) {
+        *abort_flag = 1u;
+        atomicOr(&g_device_status, 1u);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// Shared-memory matrix descriptor (K-major). layout: 0 none, 2 SW128, 4 SW64.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t sbo_bytes, uint32_t layout, uint32_t lbo_bytes) {
+  uint64_t d = (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;  // descriptor version for sm_100
+  d |= (uint64_t)layout << 61;
+  return d;
+}
+
+// Instruction descriptor of the block-scaled MMA kinds (mxf4 / mxf4nvf4): E2M1 A and B,
+// K-major, fp32 accumulate, M = 128, N = 256.
+__device__ __forceinline__ uint32_t idesc_bs(bool sparse, bool ue8m0, uint32_t sfa_id, uint32_t sfb_id) {
+  uint32_t d = 0;
+  d |= (sparse ? 1u : 0u) << 2;
+  d |= (sfb_id & 3u) << 4;
+  d |= 1u << 7;                    // A format E2M1
+  d |= 1u << 10;                   // B format E2M1
+  d |= (uint32_t)(BN >> 3) << 17;  // N
+  d |= (ue8m0 ? 1u : 0u) << 23;    // scale type: 0 UE4M3, 1 UE8M0
+  d |= (uint32_t)(BM >> 4) << 24;  // M
+  d |= (sfa_id & 3u) << 29;
+  return d;
+}
+
+template <bool MX>
+__device__ __forceinline__ void mma_dense(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                          uint32_t sfb, uint32_t acc) {
+  if (MX)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
+}
+
+template <bool MX>
+__device__ __forceinline__ void mma_sparse(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t meta, uint32_t idesc,
+                                           uint32_t sfa, uint32_t sfb, uint32_t acc) {
+  if (MX)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb), "r"(meta));
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb), "r"(meta));
+}
+
+// 32 rows x 128 bits (one 512-byte scale atom), replicated into the four lane quarters.
+__device__ __forceinline__ void tc_cp_atom(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+// 128 rows x 128 bits (metadata of 256 logical K).
+__device__ __forceinline__ void tc_cp_128x128(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// atoms of one K-tile for a scale tensor whose scale covers `span` K positions
+__host__ __device__ constexpr int atoms_per_ktile(int span) { return BK / span / 4; }
+
+template <bool MX, bool SPARSE>
+__global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const __grid_constant__ TmaMaps maps, GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
+  // bars: full[kStages], empty[kStages], acc_full, acc_empty, drain
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kStages + 3);
+  volatile uint32_t *abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t smem0 = smem_u32(smem);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+  const uint32_t acc_full = bar0 + 8u * (2 * kStages), acc_empty = acc_full + 8, drain_bar = acc_full + 16;
+
+  const int B = MX ? 32 : 16;                // dense block
+  const int span_res = B, span_sp = 2 * B;   // K positions per scale
+  const int apt_res = atoms_per_ktile(span_res), apt_sp = atoms_per_ktile(span_sp);
+  const int num_m = (p.T + BM - 1) / BM, num_n = (p.N + BN - 1) / BN, num_k = p.K / BK;
+  const int num_tiles = num_m * num_n;
+  const uint64_t limit = p.wait_limit > 0 ? (uint64_t)p.wait_limit : 4000000000ull;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.a_res) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.b) : "memory");
+    if (SPARSE) asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.a_sp) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0;       // bit s: stage s armed at least once (for the drain)
+      uint32_t last_parity = 0;  // bit s: phase parity of stage s's most recent arming
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+        const int nb_valid = min(2, (p.N_pad - n0) / 128);  // scale n-blocks inside the padded weight
+        for (int kt = 0; kt < num_k; ++kt) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, limit, abort_flag)) { ok = false; break; }
+          const uint32_t st = smem0 + stage * kStageBytes;
+          uint32_t bytes = 16384 + 32768 + apt_res * 512 + nb_valid * apt_res * 512;
+          if (SPARSE) bytes += 8192 + 2048 + apt_sp * 512 + nb_valid * apt_sp * 512;
+          mbar_expect_tx(full_bar(stage), bytes);
+          armed |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          const uint32_t fb = full_bar(stage);
+          tma_load_2d(st + OFF_ARES, &maps.a_res, kt * 128, m0, fb);
+          tma_load_2d(st + OFF_B, &maps.b, kt * 128, n0, fb);
+          const int mb = m0 / 128;
+          bulk_load(st + OFF_SFA_RES, p.sfa_res + ((size_t)mb * (p.K / span_res / 4) + (size_t)kt * apt_res) * 512,
+                    apt_res * 512, fb);
+          for (int i = 0; i < nb_valid; ++i) {
+            const int nb = n0 / 128 + i;
+            bulk_load(st + OFF_SFB_RES + i * 2048,
+                      p.sfb_dense + ((size_t)nb * (p.K / span_res / 4) + (size_t)kt * apt_res) * 512, apt_res * 512, fb);
+          }
+          if (SPARSE) {
+            tma_load_2d(st + OFF_ASP, &maps.a_sp, kt * 64, m0, fb);
+            bulk_load(st + OFF_META, p.meta + ((size_t)kt * p.T_pad + m0) * 16, 2048, fb);
+            bulk_load(st + OFF_SFA_SP, p.sfa_sp + ((size_t)mb * (p.K / span_sp / 4) + (size_t)kt * apt_sp) * 512,
+                      apt_sp * 512, fb);
+            for (int i = 0; i < nb_valid; ++i) {
+              const int nb = n0 / 128 + i;
+              bulk_load(st + OFF_SFB_SP + i * 1024,
+                        p.sfb_sparse + ((size_t)nb * (p.K / span_sp / 4) + (size_t)kt * apt_sp) * 512, apt_sp * 512,
+                        fb);
+            }
+          }
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Drain: every armed stage's most recent load completes before the CTA may exit.
+      for (int s = 0; s < kStages; ++s)
+        if (armed & (1u << s)) {
+          volatile uint32_t no_abort = 0;
+          mbar_wait(full_bar(s), (last_parity >> s) & 1u, kDrainLimitNs, &no_abort);
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      const uint32_t acc = tmem;  // lanes 0..127, columns 0..255
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(acc_empty, acc_phase ^ 1u, limit, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        for (int kt = 0; kt < num_k; ++kt) {
+          if (!mbar_wait(full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t st = smem0 + stage * kStageBytes;
+          const uint32_t sbuf = tmem + kAccCols + (kt & 1) * kScaleBufCols;
+          const uint32_t t_meta = sbuf, t_sfa_sp = sbuf + 4, t_sfa_res = sbuf + 12, t_sfb_sp = sbuf + 28,
+                         t_sfb_res = sbuf + 44;
+          // scales and metadata: shared memory -> tensor memory
+          for (int a = 0; a < apt_res; ++a) {
+            tc_cp_atom(t_sfa_res + 4 * a, sdesc(st + OFF_SFA_RES + a * 512, 128, 0, 0));
+            for (int i = 0; i < 2; ++i)
+              tc_cp_atom(t_sfb_res + 8 * a + 4 * i, sdesc(st + OFF_SFB_RES + i * 2048 + a * 512, 128, 0, 0));
+          }
+          if (SPARSE) {
+            tc_cp_128x128(t_meta, sdesc(st + OFF_META, 128, 0, 0));
+            for (int a = 0; a < apt_sp; ++a) {
+              tc_cp_atom(t_sfa_sp + 4 * a, sdesc(st + OFF_SFA_SP + a * 512, 128, 0, 0));
+              for (int i = 0; i < 2; ++i)
+                tc_cp_atom(t_sfb_sp + 8 * a + 4 * i, sdesc(st + OFF_SFB_SP + i * 1024 + a * 512, 128, 0, 0));
+            }
+          }
+          uint32_t accumulate = kt > 0 ? 1u : 0u;
+          if (SPARSE) {
+            // two sparse MMAs: 128 logical K each = 32 bytes of compressed A, 64 bytes of B
+            for (int j = 0; j < 2; ++j) {
+              const uint64_t ad = sdesc(st + OFF_ASP + 32 * j, 512, 4, 16);
+              const uint64_t bd = sdesc(st + OFF_B + 64 * j, 1024, 2, 16);
+              // NVFP4: 4 scales per row per MMA (one atom, id 0); MXFP4: 2 (half an atom)
+              const uint32_t atom = MX ? (uint32_t)(j >> 1) : (uint32_t)j;
+              const uint32_t id = MX ? (uint32_t)(2 * (j & 1)) : 0u;
+              const uint32_t sfa = (t_sfa_sp + 4 * atom) | (id << 30);
+              const uint32_t sfb = (t_sfb_sp + 8 * atom) | (id << 30);
+              mma_sparse<MX>(acc, ad, bd, t_meta + 2 * j, idesc_bs(true, MX, id, id), sfa, sfb, accumulate);
+              accumulate = 1u;
+            }
+          }
+          for (int j = 0; j < 4; ++j) {  // four dense MMAs of K = 64 (32 bytes of A and B)
+            const uint64_t ad = sdesc(st + OFF_ARES + 32 * j, 1024, 2, 16);
+            const uint64_t bd = sdesc(st + OFF_B + 32 * j, 1024, 2, 16);
+            const uint32_t atom = MX ? (uint32_t)(j >> 1) : (uint32_t)j;
+            const uint32_t id = MX ? (uint32_t)(2 * (j & 1)) : 0u;
+            const uint32_t sfa = (t_sfa_res + 4 * atom) | (id << 30);
+            const uint32_t sfb = (t_sfb_res + 8 * atom) | (id << 30);
+            mma_dense<MX>(acc, ad, bd, idesc_bs(false, MX, id, id), sfa, sfb, accumulate);
+            accumulate = 1u;
+          }
+          tc_commit(empty_bar(stage));  // frees the stage once these MMAs have read it
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+        acc_phase ^= 1u;
+      }
+      // Drain: all MMAs and copies issued above complete before TMEM is released.
+      tc_commit(drain_bar);
+      volatile uint32_t no_abort = 0;
+      mbar_wait(drain_bar, 0, kDrainLimitNs, &no_abort);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int r_local = quarter * 32 + lane;
+    uint32_t acc_phase = 0;
+    const float s_w = p.tensor_scale[0];
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+      if (!mbar_wait(acc_full, acc_phase, limit, abort_flag)) break;
+      tc_fence_after();
+      const int row = m0 + r_local;
+      const float scale = row < p.T ? __fmul_rn(p.row_scale[row], s_w) : 0.f;
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + c0, r);
+        const int col = n0 + c0;
+        if (row < p.T && col < p.N) {
+          if (p.out_f32) {
+            float *dst = reinterpret_cast<float *>(p.y) + (size_t)row * p.N + col;
+            if (col + 32 <= p.N) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4 *>(dst + i) =
+                    make_float4(__fmul_rn(__uint_as_float(r[i]), scale), __fmul_rn(__uint_as_float(r[i + 1]), scale),
+                                __fmul_rn(__uint_as_float(r[i + 2]), scale), __fmul_rn(__uint_as_float(r[i + 3]), scale));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (col + i < p.N) dst[i] = __fmul_rn(__uint_as_float(r[i]), scale);
+            }
+          } else {
+            uint32_t packed[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * i]), scale),
+                                                             __fmul_rn(__uint_as_float(r[2 * i + 1]), scale));
+              packed[i] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+            uint16_t *dst = reinterpret_cast<uint16_t *>(p.y) + (size_t)row * p.N + col;
+            if (col + 32 <= p.N) {
+#pragma unroll
+              for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<uint4 *>(dst + 2 * i) = make_uint4(packed[i], packed[i + 1], packed[i + 2], packed[i + 3]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (col + 2 * i < p.N) *reinterpret_cast<uint32_t *>(dst + 2 * i) = packed[i];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner_bytes, uint64_t rows, uint32_t box_inner,
+              uint32_t box_rows, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner_bytes, rows};
+  cuuint64_t strides[1] = {inner_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool MX, bool SPARSE>
+cudaError_t launch_t(const TmaMaps &maps, const GemmParams &p, cudaStream_t st) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(sharq_gemm_kernel<MX, SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tiles = ((p.T + BM - 1) / BM) * ((p.N + BN - 1) / BN);
+  const int grid = tiles < sms ? tiles : sms;
+  sharq_gemm_kernel<MX, SPARSE><<<grid, kThreads, kSmemBytes, st>>>(maps, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmParams &p, cudaStream_t st, const char **why) {
+  TmaMaps maps;
+  memset(&maps, 0, sizeof maps);
+  bool ok = make_map(&maps.a_res, p.a_res, (uint64_t)p.K / 2, (uint64_t)p.T, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            make_map(&maps.b, p.b, (uint64_t)p.K / 2, (uint64_t)p.N, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (ok && p.sparse)
+    ok = make_map(&maps.a_sp, p.a_sp, (uint64_t)p.K / 4, (uint64_t)p.T, 64, BM, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (!ok) {
+    *why = "cuTensorMapEncodeTiled failed (driver entry point missing or operand layout rejected)";
+    return cudaErrorInvalidValue;
+  }
+  const bool mx = p.fmt == kFmtMX;
+  if (p.sparse) return mx ? launch_t<true, true>(maps, p, st) : launch_t<false, true>(maps, p, st);
+  return mx ? launch_t<true, false>(maps, p, st) : launch_t<false, false>(maps, p, st);
+}
+
+cudaError_t read_and_clear_device_status(int *status, cudaStream_t st) {
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return e;
+  uint32_t v = 0, zero = 0;
+  if ((e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof v)) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero)) != cudaSuccess) return e;
+  *status = (int)v;
+  return cudaSuccess;
+}
+
+}  // namespace sharq

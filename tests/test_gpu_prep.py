@@ -1,0 +1,148 @@
+"""Parity of the fused preparation kernel and the dense quantizer with the CPU oracle.
+
+Without RMSNorm (the normalized input held fixed) metadata, codes and scales must be
+bit-exact. With fused RMSNorm the GPU's float64 sum of squares runs in a different order
+from the oracle's, so a row's rstd may differ by one float32 ulp: at most 1e-4 of the
+codes may then differ, each by one E2M1 step.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from oracle import sharq as O
+from tests import hwlayout as hw
+from tests.gpu_common import FMT_NAME, code_steps, f32, require_gpu, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def run_prep(S, lin, fmt, unit, use_norm, rows=None):
+    x_bits = lin.x if rows is None else lin.x[rows]
+    x = to_dev_bf16(x_bits)
+    g = to_dev_bf16(lin.gamma) if (use_norm and lin.gamma is not None) else None
+    p = S.sharq_prepare(x, g, lin.eps, 2, 4, unit, fmt)
+    torch.cuda.synchronize()
+    got = hw.read_prep(p, O.block_size(FMT_NAME[fmt]))
+    ref = O.prepare(f32(x_bits), f32(lin.gamma) if g is not None else None, lin.eps, 2, 4, unit, FMT_NAME[fmt])
+    return got, ref
+
+
+def assert_exact(got, ref):
+    for key in ("idx", "sp_codes", "sp_scales", "res_codes", "res_scales", "row_scale"):
+        a, b = got[key], ref[key]
+        assert a.shape == b.shape, (key, a.shape, b.shape)
+        if not np.array_equal(a, b):
+            bad = np.argwhere(a != b)
+            raise AssertionError(f"{key}: {len(bad)} mismatches, first at {bad[:5].tolist()}: "
+                                 f"got {a[tuple(bad[0])]} want {b[tuple(bad[0])]}")
+
+
+def assert_close_norm(got, ref):
+    assert np.array_equal(got["idx"], ref["idx"]) or np.mean(got["idx"] != ref["idx"]) <= 1e-4
+    for key in ("sp_codes", "res_codes"):
+        diff = got[key] != ref[key]
+        assert diff.mean() <= 1e-4, (key, diff.mean())
+        if diff.any():
+            assert code_steps(got[key][diff], ref[key][diff]).max() <= 1
+    for key in ("sp_scales", "res_scales"):
+        assert np.mean(got[key] != ref[key]) <= 1e-4
+    np.testing.assert_allclose(got["row_scale"], ref["row_scale"], rtol=2 ** -22)
+
+
+CASES = [  # (workload, rows) -- tiny: 64x256; ragged: 200 rows (not a multiple of 128)
+    ("tiny", None),
+    ("qkv", np.arange(200)),
+]
+
+
+def workload(name):
+    return {"tiny": wl.tiny, "qkv": lambda: wl.llama_qkv(T=256)}[name]()
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("unit", [2, 1])
+@pytest.mark.parametrize("name,rows", CASES)
+def test_prep_bit_exact_without_norm(fmt, unit, name, rows):
+    S = require_gpu()
+    got, ref = run_prep(S, workload(name), fmt, unit, use_norm=False, rows=rows)
+    assert_exact(got, ref)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("unit", [2, 1])
+@pytest.mark.parametrize("name,rows", CASES)
+def test_prep_with_fused_rmsnorm(fmt, unit, name, rows):
+    S = require_gpu()
+    got, ref = run_prep(S, workload(name), fmt, unit, use_norm=True, rows=rows)
+    assert_close_norm(got, ref)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_prep_hand_derived_rows(fmt):
+    """The golden rows of tests/golden run through the kernel (tiled to a valid K)."""
+    from tests.golden_io import load
+    S = require_gpu()
+    name = "nvfp4_pair24_row.txt" if fmt == 0 else "mxfp4_pair24_row.txt"
+    g = load(name)
+    row = (np.array(g["x_over_D"], dtype=np.float64) * g["D"]).astype(np.float32)
+    x = np.tile(row, 256 // row.size)[None, :].repeat(3, axis=0)
+    lin = wl.Linear("golden", wl.f32_to_bf16_bits(x), None, wl.f32_to_bf16_bits(np.zeros((16, 256), np.float32)))
+    got, ref = run_prep(S, lin, fmt, 2, use_norm=False)
+    assert_exact(got, ref)
+    n_sp = len(g["sp_codes"])
+    assert got["sp_codes"][0, :n_sp].tolist() == g["sp_codes"]
+    assert got["res_codes"][0, :len(g["res_codes"])].tolist() == g["res_codes"]
+
+
+def test_prep_edge_values():
+    """Zero rows, all-equal groups (ties), +-x pairs, huge and tiny values, one-token input."""
+    S = require_gpu()
+    rng = np.random.default_rng(123)
+    K = 512
+    rows = [np.zeros(K), np.ones(K), np.tile([1, -1, 1, -1], K // 4), rng.standard_normal(K) * 1e-30,
+            rng.standard_normal(K) * 3e4, np.tile([0, 0, 0, 5, 0, 0, 0, -5], K // 8),
+            np.where(np.arange(K) % 16 == 3, 300.0, 1e-3)]
+    x = wl.f32_to_bf16_bits(np.array(rows, dtype=np.float32))
+    gamma = wl.f32_to_bf16_bits(np.linspace(0.5, 1.5, K).astype(np.float32))
+    for fmt in (0, 1):
+        for unit in (1, 2):
+            lin = wl.Linear("edge", x, None, x)
+            got, ref = run_prep(S, lin, fmt, unit, use_norm=False)
+            assert_exact(got, ref)
+            lin1 = wl.Linear("one", x[4:5], gamma, x)
+            got, ref = run_prep(S, lin1, fmt, unit, use_norm=True)
+            assert_close_norm(got, ref)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_dense_quantizer_matches_oracle(fmt):
+    S = require_gpu()
+    lin = wl.llama_qkv(T=200)
+    x = to_dev_bf16(lin.x)
+    q = S.sharq_quantize_dense(x, None, lin.eps, fmt)
+    torch.cuda.synchronize()
+    B = O.block_size(FMT_NAME[fmt])
+    T, K = lin.x.shape
+    ref = O.quantize_dense(f32(lin.x), None, lin.eps, FMT_NAME[fmt])
+    assert np.array_equal(hw.unpack_e2m1(hw.to_np(q.codes), T, K), ref["codes"])
+    assert np.array_equal(hw.unswizzle_scales(hw.to_np(q.scales), T, K // B), ref["scales"])
+    assert np.array_equal(hw.to_np(q.row_scale), ref["row_scale"])
+
+
+@pytest.mark.parametrize("which,T", [("qkv", 2048), ("down", 4096)])
+def test_prep_full_size_sampled_rows(which, T):
+    """Full-size workloads in the benchmark's launch configuration; rows are independent, so
+    the oracle checks a sample of them one by one."""
+    S = require_gpu()
+    lin = wl.llama_qkv(T=T) if which == "qkv" else wl.llama_down(T=T)
+    x = to_dev_bf16(lin.x)
+    g = to_dev_bf16(lin.gamma) if lin.gamma is not None else None
+    p = S.sharq_prepare(x, g, lin.eps, 2, 4, 2, 0)
+    torch.cuda.synchronize()
+    got = hw.read_prep(p, 16)
+    rows = np.random.default_rng(0).choice(T, 48, replace=False)
+    rows = np.concatenate([rows, [0, T - 1]])
+    ref = O.prepare(f32(lin.x[rows]), f32(lin.gamma), lin.eps, 2, 4, 2, O.NVFP4)
+    sub = {k: v[rows] for k, v in got.items()}
+    (assert_close_norm if g is not None else assert_exact)(sub, ref)
