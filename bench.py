@@ -212,9 +212,17 @@ def run_sharq(args, rank, world, local):
     torch.cuda.synchronize()
     assert S.sharq_device_status() == S.SHARQ_OK
 
-    # ---- device-timed whole steps
+    # ---- device-timed whole steps; the clock sampler runs from a 1 s pre-roll of the same
+    # step (nvidia-smi needs ~100 ms per sample) through the timed region
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
+        t_end = time.perf_counter() + 1.0
+        i = 0
+        while time.perf_counter() < t_end:
+            step(i)
+            i += 1
+            if i % 64 == 0:
+                torch.cuda.synchronize()
         barrier(world)
         torch.cuda.synchronize()
         ev0.record(stream)
@@ -333,6 +341,29 @@ def run_sharq(args, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(args):
+    """A few launches of one kernel on the QKV shape with ``--tokens`` rows (for ncu captures)."""
+    import fp4_activation_sparse_b200 as S
+    lin = wl.llama_qkv(T=args.tokens)
+    T, K, N = lin.shape
+    x, g, w = to_dev(lin.x), to_dev(lin.gamma), to_dev(lin.w)
+    wp = S.sharq_pack_weight(w, "nvfp4")
+    p = S.sharq_prepare(x, g, lin.eps)
+    q = S.sharq_quantize_dense(x, g, lin.eps)
+    y = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        if args.profile == "prep":
+            S.sharq_prepare(x, g, lin.eps, out=p)
+        elif args.profile == "linear":
+            S.sharq_linear(p, wp, y=y)
+        elif args.profile == "dense":
+            S.sharq_quantize_dense(x, g, lin.eps, out=q)
+            S.sharq_linear_dense(q, wp, y=y)
+    torch.cuda.synchronize()
+    assert S.sharq_device_status() == S.SHARQ_OK
+    print(json.dumps({"profile": args.profile, "tokens": T, "k": K, "n": N}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -340,7 +371,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sharq", "reference"], default="sharq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["prep", "linear", "dense"], help="run 3 launches of one kernel for ncu")
+    ap.add_argument("--tokens", type=int, default=2048)
     args = ap.parse_args()
+    if args.profile:
+        run_profile(args)
+        return
     rank, world, local = dist_setup(args.gpus)
     try:
         if args.impl == "reference":

@@ -63,7 +63,7 @@ size_t sharq_prep_buffer_sizes(int tokens, int k, int nm_n, int nm_m, int unit, 
   if (!sizes) { fail(SHARQ_ERR_INVALID_ARG, "sizes is null"); return 0; }
   if (!valid_fmt(fmt)) { fail(SHARQ_ERR_INVALID_ARG, "unknown fmt %d", fmt); return 0; }
   if (check_shape(tokens, k, "tokens") || check_pattern(nm_n, nm_m, unit)) return 0;
-  const size_t T = tokens, K = k, Tp = sharq::round_up(tokens, 128), B = block_of(fmt);
+  const size_t T = tokens, K = k, Tp = sharq::round_up(tokens, 256), B = block_of(fmt);
   const size_t stored = K * nm_n / nm_m;
   const size_t slab_span = 32u * nm_m * unit;
   sizes[0] = T * stored / 2;            // sparse codes
@@ -123,7 +123,9 @@ static int prepare_common(const void *x, int tokens, int k, const void *gamma, f
   if (!x) return fail(SHARQ_ERR_INVALID_ARG, "x is null");
   if (!valid_fmt(fmt)) return fail(SHARQ_ERR_INVALID_ARG, "unknown fmt %d", fmt);
   if (int s = check_shape(tokens, k, "tokens")) return s;
-  if (!aligned16(x) || (gamma && !aligned16(gamma))) return fail(SHARQ_ERR_INVALID_ARG, "x/gamma must be 16-byte aligned");
+  if (k > 32768) return fail(SHARQ_ERR_INVALID_ARG, "k must be <= 32768 for the preparation kernel (got %d)", k);
+  if (((uintptr_t)x & 31u) || ((uintptr_t)gamma & 31u))
+    return fail(SHARQ_ERR_INVALID_ARG, "x and gamma must be 32-byte aligned (256-bit loads)");
   if (!res_codes || !res_scales || !row_scale) return fail(SHARQ_ERR_INVALID_ARG, "null output buffer");
   if (!dense && (!sp_codes || !meta || !sp_scales)) return fail(SHARQ_ERR_INVALID_ARG, "null output buffer");
   const void *bufs[6] = {sp_codes, meta, sp_scales, res_codes, res_scales, row_scale};
@@ -136,7 +138,7 @@ static int prepare_common(const void *x, int tokens, int k, const void *gamma, f
   p.eps = eps;
   p.T = tokens;
   p.K = k;
-  p.T_pad = sharq::round_up(tokens, 128);
+  p.T_pad = sharq::round_up(tokens, 256);
   p.sp_codes = sp_codes;
   p.meta = meta;
   p.sp_scales = sp_scales;
@@ -234,7 +236,7 @@ int sharq_linear(const sharq_prep *a, const sharq_wpack *w, void *y, int out_dty
   g.T = a->tokens;
   g.N = w->n_out;
   g.K = a->k;
-  g.T_pad = sharq::round_up(a->tokens, 128);
+  g.T_pad = sharq::round_up(a->tokens, 256);
   g.N_pad = sharq::round_up(w->n_out, 128);
   g.fmt = a->fmt;
   g.out_f32 = out_dtype == SHARQ_OUT_F32;
@@ -264,7 +266,7 @@ int sharq_linear_dense(const void *codes, const void *scales, const float *row_s
   g.T = tokens;
   g.N = w->n_out;
   g.K = k;
-  g.T_pad = sharq::round_up(tokens, 128);
+  g.T_pad = sharq::round_up(tokens, 256);
   g.N_pad = sharq::round_up(w->n_out, 128);
   g.fmt = w->fmt;
   g.out_f32 = out_dtype == SHARQ_OUT_F32;

@@ -7,20 +7,23 @@
 // error. The two paths share a single FP4 weight payload with path-specific scale
 // views." The README ("Benchmarks") enables "epilogue fusion" on this path.
 //
-// sm_100a design (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0       TMA producer: per K-tile of 256 it loads the residual codes (SW128),
-//                the compressed backbone codes (SW64), the weight codes (SW128), the
-//                backbone metadata and the four scale tiles (1-D bulk copies of
-//                pre-tiled 128x4 atoms). Each weight tile is loaded once and feeds
-//                both MMAs.
-//   warp 1       TMEM owner and MMA issuer: tcgen05.cp moves scales and metadata to
-//                tensor memory, then two tcgen05.mma.sp (K=128 logical, pairwise 4:8)
-//                and four dense tcgen05.mma (K=64) accumulate into one 128x256 fp32
-//                accumulator. Both paths carry the same per-row scale s_x, so one
-//                accumulator holds their sum.
-//   warps 2..5   epilogue: tcgen05.ld, y = acc * s_x[row] * s_w, bf16/fp32 stores.
-// Every mbarrier wait is bounded by a time limit; on expiry the CTA records a status
-// word, stops issuing, waits (bounded) for its own copies and MMAs, frees TMEM and exits.
+// sm_100a design. A cluster of two CTAs on the two SMs of a TPC works on one 256 x 256
+// output tile with cta_group::2 MMAs (M = 256, N = 256): each CTA loads its own 128
+// activation rows and half of the weight tile (128 rows), so every weight byte crosses
+// into shared memory once per pair. Persistent over tiles, K-tiles of 256, four stages.
+//   warp 0      TMA producer (both CTAs): residual codes (SW128), compressed backbone codes
+//               (SW64), weight codes (SW128), backbone metadata and the four scale tiles
+//               (pre-tiled 128x4 atoms); every load completes on the leader CTA's barrier.
+//               Each weight tile feeds both MMAs.
+//   warp 1      TMEM owner (both CTAs) and, in the leader, the single MMA-issuing thread:
+//               tcgen05.cp moves scales and metadata to tensor memory, then two
+//               tcgen05.mma.sp (K=128 logical, pairwise 4:8) and four dense tcgen05.mma
+//               (K=64) accumulate into one fp32 accumulator of 128 x 256 per CTA. Both
+//               paths carry the same per-row scale s_x, so one accumulator holds their sum.
+//               Commits arrive on both CTAs' barriers (multicast commit).
+//   warps 2..9  epilogue (both CTAs): tcgen05.ld, y = acc * s_x[row] * s_w, bf16/fp32 stores.
+// Every mbarrier wait is bounded by a time limit; on expiry the CTA records a status word,
+// stops issuing, drains (bounded) what it issued, frees TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -35,9 +38,13 @@ __device__ uint32_t g_device_status = 0;  // bit 0: a bounded wait gave up
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 256;  // BK in logical K elements
-constexpr int kStages = 3;
-constexpr int kThreads = 192;
+constexpr int BM = 128;   // activation rows per CTA (256 per pair)
+constexpr int BN = 256;   // output columns per pair tile
+constexpr int BNH = 128;  // weight rows loaded per CTA
+constexpr int BK = 256;   // logical K per stage
+constexpr int kStages = 4;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = 256;
 constexpr uint32_t kScaleBufCols = 80;  // per K-tile parity: meta 4, SFA_sp 8, SFA_res 16, SFB_sp 16, SFB_res 32
@@ -45,25 +52,42 @@ constexpr uint32_t kScaleBufCols = 80;  // per K-tile parity: meta 4, SFA_sp 8, 
 // test lowers the limit of the ordinary waits.
 constexpr uint64_t kDrainLimitNs = 4000000000ull;
 
-// shared-memory stage layout (bytes)
-constexpr int OFF_ARES = 0;       // 128 rows x 128 B, SW128
-constexpr int OFF_B = 16384;      // 256 rows x 128 B, SW128
-constexpr int OFF_ASP = 49152;    // 128 rows x 64 B, SW64
-constexpr int OFF_META = 57344;   // 128 rows x 16 B
-constexpr int OFF_SFA_RES = 59392;
-constexpr int OFF_SFA_SP = 61440;
-constexpr int OFF_SFB_RES = 62464;  // n-block 0 at +0, n-block 1 at +2048
-constexpr int OFF_SFB_SP = 66560;   // n-block 0 at +0, n-block 1 at +1024
-constexpr int kStageBytes = 68608;
+// shared-memory stage layout (bytes), identical in both CTAs
+constexpr int OFF_ARES = 0;         // 128 rows x 128 B, SW128
+constexpr int OFF_B = 16384;        // 128 weight rows x 128 B, SW128
+constexpr int OFF_ASP = 32768;      // 128 rows x 64 B, SW64
+constexpr int OFF_META = 40960;     // 128 rows x 16 B
+constexpr int OFF_SFA_RES = 43008;  // up to 4 atoms
+constexpr int OFF_SFA_SP = 45056;   // up to 2 atoms
+constexpr int OFF_SFB_RES = 46080;  // n-block 0 at +0, n-block 1 at +2048
+constexpr int OFF_SFB_SP = 50176;   // n-block 0 at +0, n-block 1 at +1024
+constexpr int kStageBytes = 52224;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align slack*/ + 256 /*barriers*/;
 
 struct __align__(64) TmaMaps {
-  CUtensorMap a_res, a_sp, b;
+  CUtensorMap a_res, a_sp, b, meta, sfa_res, sfa_sp, sfb_res, sfb_sp;
 };
 
 // ---------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// address of the same shared-memory offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -74,14 +98,16 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+// arrive on a barrier given by its shared::cluster address (own or peer CTA)
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
       : "memory");
@@ -113,25 +139,33 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
   }
 }
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          dst),
-      "l"(map), "r"(c0), "r"(c1), "r"(bar)
-      : "memory");
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+  const uint64_t t0 = globaltimer();
+  while (globaltimer() - t0 < ns) {
+  }
 }
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
+// 2-D TMA load into this CTA's shared memory, completing on the barrier at `bar_cluster`
+// (the leader CTA's barrier) -- the cta_group::2 form lets either CTA of the pair signal it.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                            uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(bar_cluster)
+      : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+// arrive once on the barrier at the same offset in both CTAs when this thread's MMAs finish
+__device__ __forceinline__ void tc_commit_both(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
 }
 
 // Shared-memory matrix descriptor (K-major). layout: 0 none, 2 SW128, 4 SW64.
@@ -145,16 +179,16 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t sbo_bytes, uin
 }
 
 // Instruction descriptor of the block-scaled MMA kinds (mxf4 / mxf4nvf4): E2M1 A and B,
-// K-major, fp32 accumulate, M = 128, N = 256.
+// K-major, fp32 accumulate, M = 256 (two CTAs), N = 256.
 __device__ __forceinline__ uint32_t idesc_bs(bool sparse, bool ue8m0, uint32_t sfa_id, uint32_t sfb_id) {
   uint32_t d = 0;
   d |= (sparse ? 1u : 0u) << 2;
   d |= (sfb_id & 3u) << 4;
-  d |= 1u << 7;                    // A format E2M1
-  d |= 1u << 10;                   // B format E2M1
-  d |= (uint32_t)(BN >> 3) << 17;  // N
-  d |= (ue8m0 ? 1u : 0u) << 23;    // scale type: 0 UE4M3, 1 UE8M0
-  d |= (uint32_t)(BM >> 4) << 24;  // M
+  d |= 1u << 7;                          // A format E2M1
+  d |= 1u << 10;                         // B format E2M1
+  d |= (uint32_t)(BN >> 3) << 17;        // N
+  d |= (ue8m0 ? 1u : 0u) << 23;          // scale type: 0 UE4M3, 1 UE8M0
+  d |= (uint32_t)((2 * BM) >> 4) << 24;  // M
   d |= (sfa_id & 3u) << 29;
   return d;
 }
@@ -165,12 +199,12 @@ __device__ __forceinline__ void mma_dense(uint32_t d_tmem, uint64_t a, uint64_t 
   if (MX)
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
   else
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
             d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
 }
@@ -181,25 +215,26 @@ __device__ __forceinline__ void mma_sparse(uint32_t d_tmem, uint64_t a, uint64_t
   if (MX)
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.sp.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}" ::"r"(
+        "tcgen05.mma.sp.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}" ::"r"(
             d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb), "r"(meta));
   else
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.sp.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}" ::"r"(
+        "tcgen05.mma.sp.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}" ::"r"(
             d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb), "r"(meta));
 }
 
-// 32 rows x 128 bits (one 512-byte scale atom), replicated into the four lane quarters.
+// 32 rows x 128 bits (one 512-byte scale atom), replicated into the four lane quarters;
+// issued by the leader, performed in both CTAs from their own shared memory.
 __device__ __forceinline__ void tc_cp_atom(uint32_t taddr, uint64_t desc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
 
-// 128 rows x 128 bits (metadata of 256 logical K).
+// 128 rows x 128 bits (metadata of 256 logical K), in both CTAs.
 __device__ __forceinline__ void tc_cp_128x128(uint32_t taddr, uint64_t desc) {
-  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+  asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
@@ -218,7 +253,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
 __host__ __device__ constexpr int atoms_per_ktile(int span) { return BK / span / 4; }
 
 template <bool MX, bool SPARSE>
-__global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const __grid_constant__ TmaMaps maps, GemmParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    sharq_gemm_kernel(const __grid_constant__ TmaMaps maps, GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
@@ -227,17 +263,20 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const __grid_co
   volatile uint32_t *abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
   const uint32_t smem0 = smem_u32(smem);
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
   const uint32_t acc_full = bar0 + 8u * (2 * kStages), acc_empty = acc_full + 8, drain_bar = acc_full + 16;
 
-  const int B = MX ? 32 : 16;                // dense block
-  const int span_res = B, span_sp = 2 * B;   // K positions per scale
+  const int B = MX ? 32 : 16;               // dense block
+  const int span_res = B, span_sp = 2 * B;  // K positions per scale
   const int apt_res = atoms_per_ktile(span_res), apt_sp = atoms_per_ktile(span_sp);
-  const int num_m = (p.T + BM - 1) / BM, num_n = (p.N + BN - 1) / BN, num_k = p.K / BK;
+  const int num_m = (p.T + 2 * BM - 1) / (2 * BM), num_n = (p.N + BN - 1) / BN, num_k = p.K / BK;
   const int num_tiles = num_m * num_n;
+  const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
   const uint64_t limit = p.wait_limit > 0 ? (uint64_t)p.wait_limit : 4000000000ull;
 
   if (threadIdx.x == 0) {
@@ -246,84 +285,97 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const __grid_co
       mbar_init(empty_bar(s), 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    mbar_init(acc_empty, 2 * kEpiWarps);
     mbar_init(drain_bar, 1);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.a_res) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.b) : "memory");
-    if (SPARSE) asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.a_sp) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.sfa_res) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.sfb_res) : "memory");
+    if (SPARSE) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.a_sp) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.meta) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.sfa_sp) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.sfb_sp) : "memory");
+    }
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // barriers initialized and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t armed = 0;       // bit s: stage s armed at least once (for the drain)
-      uint32_t last_parity = 0;  // bit s: phase parity of stage s's most recent arming
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
-        const int nb_valid = min(2, (p.N_pad - n0) / 128);  // scale n-blocks inside the padded weight
+      uint32_t armed = 0, last_parity = 0;  // bit s: stage s armed / its last phase parity
+      bool issued = false, ok = true;
+      const uint32_t full_leader0 = map_to_rank(full_bar(0), 0);
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        const int m0 = (tile % num_m) * (2 * BM) + (int)rank * BM;  // this CTA's activation rows
+        const int n0 = (tile / num_m) * BN;                          // the pair's output columns
+        const int nb_valid = min(2, (p.N_pad - n0) / 128);            // scale n-blocks inside the padded weight
+        const int mb = m0 / 128;
         for (int kt = 0; kt < num_k; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, limit, abort_flag)) { ok = false; break; }
           const uint32_t st = smem0 + stage * kStageBytes;
-          uint32_t bytes = 16384 + 32768 + apt_res * 512 + nb_valid * apt_res * 512;
-          if (SPARSE) bytes += 8192 + 2048 + apt_sp * 512 + nb_valid * apt_sp * 512;
-          mbar_expect_tx(full_bar(stage), bytes);
-          armed |= 1u << stage;
-          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          const uint32_t fb = full_bar(stage);
-          tma_load_2d(st + OFF_ARES, &maps.a_res, kt * 128, m0, fb);
-          tma_load_2d(st + OFF_B, &maps.b, kt * 128, n0, fb);
-          const int mb = m0 / 128;
-          bulk_load(st + OFF_SFA_RES, p.sfa_res + ((size_t)mb * (p.K / span_res / 4) + (size_t)kt * apt_res) * 512,
-                    apt_res * 512, fb);
-          for (int i = 0; i < nb_valid; ++i) {
-            const int nb = n0 / 128 + i;
-            bulk_load(st + OFF_SFB_RES + i * 2048,
-                      p.sfb_dense + ((size_t)nb * (p.K / span_res / 4) + (size_t)kt * apt_res) * 512, apt_res * 512, fb);
+          if (leader) {
+            uint32_t bytes = 16384 + 16384 + apt_res * 512 + nb_valid * apt_res * 512;
+            if (SPARSE) bytes += 8192 + 2048 + apt_sp * 512 + nb_valid * apt_sp * 512;
+            mbar_expect_tx(full_bar(stage), 2 * bytes);
+            armed |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           }
+          const uint32_t fb = full_leader0 + 8u * stage;
+          tma_load_2d(st + OFF_ARES, &maps.a_res, kt * 128, m0, fb);
+          tma_load_2d(st + OFF_B, &maps.b, kt * 128, n0 + (int)rank * BNH, fb);
+          tma_load_2d(st + OFF_SFA_RES, &maps.sfa_res, 0, mb * (p.K / span_res / 4) + kt * apt_res, fb);
+          for (int i = 0; i < nb_valid; ++i)
+            tma_load_2d(st + OFF_SFB_RES + i * 2048, &maps.sfb_res, 0,
+                        (n0 / 128 + i) * (p.K / span_res / 4) + kt * apt_res, fb);
           if (SPARSE) {
             tma_load_2d(st + OFF_ASP, &maps.a_sp, kt * 64, m0, fb);
-            bulk_load(st + OFF_META, p.meta + ((size_t)kt * p.T_pad + m0) * 16, 2048, fb);
-            bulk_load(st + OFF_SFA_SP, p.sfa_sp + ((size_t)mb * (p.K / span_sp / 4) + (size_t)kt * apt_sp) * 512,
-                      apt_sp * 512, fb);
-            for (int i = 0; i < nb_valid; ++i) {
-              const int nb = n0 / 128 + i;
-              bulk_load(st + OFF_SFB_SP + i * 1024,
-                        p.sfb_sparse + ((size_t)nb * (p.K / span_sp / 4) + (size_t)kt * apt_sp) * 512, apt_sp * 512,
-                        fb);
-            }
+            tma_load_2d(st + OFF_META, &maps.meta, 0, kt * p.T_pad + m0, fb);
+            tma_load_2d(st + OFF_SFA_SP, &maps.sfa_sp, 0, mb * (p.K / span_sp / 4) + kt * apt_sp, fb);
+            for (int i = 0; i < nb_valid; ++i)
+              tma_load_2d(st + OFF_SFB_SP + i * 1024, &maps.sfb_sp, 0,
+                          (n0 / 128 + i) * (p.K / span_sp / 4) + kt * apt_sp, fb);
           }
+          issued = true;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
-      // Drain: every armed stage's most recent load completes before the CTA may exit.
-      for (int s = 0; s < kStages; ++s)
-        if (armed & (1u << s)) {
-          volatile uint32_t no_abort = 0;
-          mbar_wait(full_bar(s), (last_parity >> s) & 1u, kDrainLimitNs, &no_abort);
+      if (!ok) {
+        // Drain before exit: the leader sees every phase it armed complete (its own and the
+        // peer's bytes); the peer cannot observe the leader's barrier, so it lets its loads land.
+        if (leader) {
+          for (int s = 0; s < kStages; ++s)
+            if (armed & (1u << s)) {
+              volatile uint32_t no_abort = 0;
+              mbar_wait(full_bar(s), (last_parity >> s) & 1u, kDrainLimitNs, &no_abort);
+            }
+        } else if (issued) {
+          spin_ns(200000);
         }
+      }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (leader CTA)
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      const uint32_t acc = tmem;  // lanes 0..127, columns 0..255
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const uint32_t acc = tmem;  // lanes 0..127 of each CTA, columns 0..255
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
         if (!mbar_wait(acc_empty, acc_phase ^ 1u, limit, abort_flag)) { ok = false; break; }
         tc_fence_after();
         for (int kt = 0; kt < num_k; ++kt) {
@@ -333,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const __grid_co
           const uint32_t sbuf = tmem + kAccCols + (kt & 1) * kScaleBufCols;
           const uint32_t t_meta = sbuf, t_sfa_sp = sbuf + 4, t_sfa_res = sbuf + 12, t_sfb_sp = sbuf + 28,
                          t_sfb_res = sbuf + 44;
-          // scales and metadata: shared memory -> tensor memory
+          // scales and metadata: shared memory -> tensor memory (both CTAs)
           for (int a = 0; a < apt_res; ++a) {
             tc_cp_atom(t_sfa_res + 4 * a, sdesc(st + OFF_SFA_RES + a * 512, 128, 0, 0));
             for (int i = 0; i < 2; ++i)
@@ -372,31 +424,33 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const __grid_co
             mma_dense<MX>(acc, ad, bd, idesc_bs(false, MX, id, id), sfa, sfb, accumulate);
             accumulate = 1u;
           }
-          tc_commit(empty_bar(stage));  // frees the stage once these MMAs have read it
+          tc_commit_both(empty_bar(stage));  // frees the stage in both CTAs once these MMAs have read it
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        tc_commit_both(acc_full);
         acc_phase ^= 1u;
       }
       // Drain: all MMAs and copies issued above complete before TMEM is released.
-      tc_commit(drain_bar);
+      tc_commit_both(drain_bar);
       volatile uint32_t no_abort = 0;
       mbar_wait(drain_bar, 0, kDrainLimitNs, &no_abort);
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
-    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    // ------------------------------------------------------------ epilogue (warps 2..9, both CTAs)
+    const int quarter = warp & 3;          // TMEM lane quarter this warp may access
+    const int col_half = (warp - 2) >> 2;  // columns [128*col_half, 128*col_half + 128)
     const int r_local = quarter * 32 + lane;
+    const uint32_t acc_empty_leader = map_to_rank(acc_empty, 0);
     uint32_t acc_phase = 0;
     const float s_w = p.tensor_scale[0];
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+      const int m0 = (tile % num_m) * (2 * BM) + (int)rank * BM, n0 = (tile / num_m) * BN;
       if (!mbar_wait(acc_full, acc_phase, limit, abort_flag)) break;
       tc_fence_after();
       const int row = m0 + r_local;
       const float scale = row < p.T ? __fmul_rn(p.row_scale[row], s_w) : 0.f;
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = col_half * 128; c0 < col_half * 128 + 128; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + c0, r);
         const int col = n0 + c0;
@@ -437,15 +491,17 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const __grid_co
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
       acc_phase ^= 1u;
     }
   }
 
+  // Both CTAs: the leader arrives here only after its MMAs drained, so neither CTA frees
+  // tensor memory the pair's MMAs still write, and no remote arrive targets an exited CTA.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
 // ---------------------------------------------------------------- host side
@@ -462,17 +518,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-bool make_map(CUtensorMap *m, const void *base, uint64_t inner_bytes, uint64_t rows, uint32_t box_inner,
-              uint32_t box_rows, CUtensorMapSwizzle sw) {
+// 2-D map over `rows` rows of `inner` elements (uint8 or uint32), box `box_inner` x `box_rows`.
+bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t inner, uint64_t rows,
+              uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {inner_bytes, rows};
-  cuuint64_t strides[1] = {inner_bytes};
+  const uint64_t esz = dt == CU_TENSOR_MAP_DATA_TYPE_UINT32 ? 4 : 1;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * esz};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <bool MX, bool SPARSE>
@@ -487,9 +544,9 @@ cudaError_t launch_t(const TmaMaps &maps, const GemmParams &p, cudaStream_t st) 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int tiles = ((p.T + BM - 1) / BM) * ((p.N + BN - 1) / BN);
-  const int grid = tiles < sms ? tiles : sms;
-  sharq_gemm_kernel<MX, SPARSE><<<grid, kThreads, kSmemBytes, st>>>(maps, p);
+  const int tiles = ((p.T + 2 * BM - 1) / (2 * BM)) * ((p.N + BN - 1) / BN);
+  const int pairs = tiles < sms / 2 ? tiles : sms / 2;
+  sharq_gemm_kernel<MX, SPARSE><<<2 * pairs, kThreads, kSmemBytes, st>>>(maps, p);
   return cudaGetLastError();
 }
 
@@ -498,10 +555,21 @@ cudaError_t launch_t(const TmaMaps &maps, const GemmParams &p, cudaStream_t st) 
 cudaError_t launch_gemm(const GemmParams &p, cudaStream_t st, const char **why) {
   TmaMaps maps;
   memset(&maps, 0, sizeof maps);
-  bool ok = make_map(&maps.a_res, p.a_res, (uint64_t)p.K / 2, (uint64_t)p.T, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            make_map(&maps.b, p.b, (uint64_t)p.K / 2, (uint64_t)p.N, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8, U32 = CU_TENSOR_MAP_DATA_TYPE_UINT32;
+  const auto NONE = CU_TENSOR_MAP_SWIZZLE_NONE;
+  const int B = p.fmt == kFmtMX ? 32 : 16;
+  const uint64_t atoms_res_a = (uint64_t)(p.T_pad / 128) * (p.K / B / 4);
+  const uint64_t atoms_res_b = (uint64_t)(p.N_pad / 128) * (p.K / B / 4);
+  const uint32_t apt_res = atoms_per_ktile(B), apt_sp = atoms_per_ktile(2 * B);
+  bool ok = make_map(&maps.a_res, p.a_res, U8, (uint64_t)p.K / 2, (uint64_t)p.T, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            make_map(&maps.b, p.b, U8, (uint64_t)p.K / 2, (uint64_t)p.N, 128, BNH, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            make_map(&maps.sfa_res, p.sfa_res, U32, 128, atoms_res_a, 128, apt_res, NONE) &&
+            make_map(&maps.sfb_res, p.sfb_dense, U32, 128, atoms_res_b, 128, apt_res, NONE);
   if (ok && p.sparse)
-    ok = make_map(&maps.a_sp, p.a_sp, (uint64_t)p.K / 4, (uint64_t)p.T, 64, BM, CU_TENSOR_MAP_SWIZZLE_64B);
+    ok = make_map(&maps.a_sp, p.a_sp, U8, (uint64_t)p.K / 4, (uint64_t)p.T, 64, BM, CU_TENSOR_MAP_SWIZZLE_64B) &&
+         make_map(&maps.meta, p.meta, U32, 4, (uint64_t)(p.K / 256) * p.T_pad, 4, BM, NONE) &&
+         make_map(&maps.sfa_sp, p.sfa_sp, U32, 128, atoms_res_a / 2, 128, apt_sp, NONE) &&
+         make_map(&maps.sfb_sp, p.sfb_sparse, U32, 128, atoms_res_b / 2, 128, apt_sp, NONE);
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or operand layout rejected)";
     return cudaErrorInvalidValue;

@@ -6,25 +6,28 @@
 // defined "relative to the quantized sparse backbone rather than the
 // unquantized sparse values".
 //
-// One pass over the bf16 activations. A team of threads owns one token row; each
-// thread owns chunks of 64 consecutive K elements (128 bytes of input). The row's
-// sum of squares (RMSNorm, float64) and amax (second-level scale) are team
-// reductions; everything else is local to the chunk:
-//   mask (per group of 8 for pairs / 4 for elements) -> 32 stored values ->
-//   backbone blocks (2 x 16 NVFP4 / 1 x 32 MXFP4) -> dequantized backbone ->
-//   residual -> residual blocks (4 x 16 / 2 x 32).
-// The outputs go straight to the layouts the GEMM's TMA and tensor-core scale copies
-// read, so no re-layout pass follows. Float32 operations use explicit _rn
-// intrinsics so no contraction changes a rounding.
+// One read of the bf16 activations. A team of W warps owns one token row (W = K/4096
+// rounded up); every lane owns "double pieces" of 16 consecutive K elements (one 256-bit
+// load), consecutive lanes owning consecutive pieces, and keeps its whole share of the
+// row in registers. Passes over those registers: sum of squares (RMSNorm), row amax
+// (second-level scale), then per double piece:
+//   mask (2 groups of 4 pairs / 4 groups of 4 elements) -> backbone block amax (the
+//   largest element of a group is always kept, so it is the max of group maxima) ->
+//   backbone codes for every element with the backbone block scale; the kept bytes are
+//   stored, the dropped ones zeroed -> dequantized backbone -> residual r = xh - deq ->
+//   residual block scale and codes.
+// Blocks spanning lanes reduce with warp shuffles; scale and metadata bytes are gathered
+// by shuffles into whole 32-bit words, so every store is coalesced. Float32 arithmetic
+// uses explicit round-to-nearest operations, so no contraction changes a rounding.
 #include "sharq_common.cuh"
 #include "sharq_internal.h"
-#include "sharq_quant.cuh"
 
 namespace sharq {
 
 namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
+constexpr int kMaxDP = 8;  // double pieces (16 elements) per lane
 
 // mask of kept units (bit i = unit i kept) -> metadata nibble i0 | i1 << 2
 constexpr unsigned long long kNibbleLut =
@@ -32,7 +35,7 @@ constexpr unsigned long long kNibbleLut =
     (13ull << (10 * 4)) | (14ull << (12 * 4));
 
 // Top-2 of four keys, ties to the lower index: the two units whose rank
-// (#keys strictly above + #equal keys at lower index) is below 2.
+// (#keys strictly above + #equal keys at a lower index) is below 2.
 __device__ __forceinline__ uint32_t top2_of_4(float k0, float k1, float k2, float k3) {
   int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
   if (k0 >= k1) ++r1; else ++r0;
@@ -45,192 +48,286 @@ __device__ __forceinline__ uint32_t top2_of_4(float k0, float k1, float k2, floa
   return (uint32_t)(kNibbleLut >> (m * 4)) & 0xFu;
 }
 
-__device__ __forceinline__ float sel4(uint32_t i, float a, float b, float c, float d) {
-  return i == 0 ? a : (i == 1 ? b : (i == 2 ? c : d));
+// ---------------------------------------------------------------- float32 pairs
+// Element-wise round-to-nearest products / differences of two lanes. (Scalar operations:
+// the packed f32x2 forms were measured not to round like these on every input.)
+__device__ __forceinline__ void mul2(float &a0, float &a1, float b0, float b1) {
+  a0 = __fmul_rn(a0, b0);
+  a1 = __fmul_rn(a1, b1);
+}
+__device__ __forceinline__ void sub2(float &a0, float &a1, float b0, float b1) {
+  a0 = __fsub_rn(a0, b0);
+  a1 = __fsub_rn(a1, b1);
 }
 
-// ---------------------------------------------------------------- team reductions
-// Butterfly reductions: every lane ends with the identical result (each step adds
-// the same two operands), so all threads of a row derive bit-identical scales.
-template <typename V>
-__device__ __forceinline__ V team_sum(V v, int TS, V *sm) {
-  const int lim = TS < 32 ? TS : 32;
-  for (int o = lim >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
-  if (TS > 32) {
-    const int w = threadIdx.x >> 5, nw = TS >> 5;
-    if ((threadIdx.x & 31) == 0) sm[w] = v;
-    __syncthreads();
-    v = sm[0];
-    for (int i = 1; i < nw; ++i) v += sm[i];
-    __syncthreads();
-  }
-  return v;
+// ---------------------------------------------------------------- I/O
+__device__ __forceinline__ void ld256(const void *p, uint32_t (&r)[8]) {
+  asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "l"(p));
 }
 
-__device__ __forceinline__ float team_max(float v, int TS, float *sm) {
-  const int lim = TS < 32 ? TS : 32;
-  for (int o = lim >> 1; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
-  if (TS > 32) {
-    const int w = threadIdx.x >> 5, nw = TS >> 5;
-    if ((threadIdx.x & 31) == 0) sm[w] = v;
-    __syncthreads();
-    v = sm[0];
-    for (int i = 1; i < nw; ++i) v = fmaxf(v, sm[i]);
-    __syncthreads();
-  }
-  return v;
-}
-
-// ---------------------------------------------------------------- chunk I/O
-__device__ __forceinline__ void load_bf16x64(const uint16_t *src, float *v) {
-  const uint4 *s = reinterpret_cast<const uint4 *>(src);
+__device__ __forceinline__ void unpack16(const uint32_t (&w)[8], float *v) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint4 q = __ldg(s + i);
-    v[8 * i + 0] = bf16lo(q.x); v[8 * i + 1] = bf16hi(q.x);
-    v[8 * i + 2] = bf16lo(q.y); v[8 * i + 3] = bf16hi(q.y);
-    v[8 * i + 4] = bf16lo(q.z); v[8 * i + 5] = bf16hi(q.z);
-    v[8 * i + 6] = bf16lo(q.w); v[8 * i + 7] = bf16hi(q.w);
+    v[2 * i] = bf16lo(w[i]);
+    v[2 * i + 1] = bf16hi(w[i]);
   }
 }
 
-__device__ __forceinline__ void apply_norm(float *v, const uint16_t *gamma, float rstd) {
-  const uint4 *g = reinterpret_cast<const uint4 *>(gamma);
+// xh = fp32(fp32(x * rstd) * gamma) for 16 values
+__device__ __forceinline__ void normalize16(float *v, const uint16_t *gamma16, float rstd) {
+  uint32_t g[8];
+  ld256(gamma16, g);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint4 q = __ldg(g + i);
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      v[8 * i + 2 * j] = __fmul_rn(__fmul_rn(v[8 * i + 2 * j], rstd), bf16lo(w[j]));
-      v[8 * i + 2 * j + 1] = __fmul_rn(__fmul_rn(v[8 * i + 2 * j + 1], rstd), bf16hi(w[j]));
-    }
+    mul2(v[2 * i], v[2 * i + 1], rstd, rstd);
+    mul2(v[2 * i], v[2 * i + 1], bf16lo(g[i]), bf16hi(g[i]));
   }
 }
 
-// ---------------------------------------------------------------- one chunk
-// Quantizes the 64 values v[] (already normalized) of chunk `c` of row `row`.
+// Gather byte b of lanes (lane, lane+d, lane+2d, lane+3d) into one word (valid on the first).
+__device__ __forceinline__ uint32_t gather4(uint32_t b, int d) {
+  const uint32_t b1 = __shfl_down_sync(kFull, b, d);
+  const uint32_t b2 = __shfl_down_sync(kFull, b, 2 * d);
+  const uint32_t b3 = __shfl_down_sync(kFull, b, 3 * d);
+  return (b & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
+}
+
+// ---------------------------------------------------------------- block scales
+// NVFP4: E4M3 code of fp32(amax*g); d = fp32(dec*s); inv = 1/d (0 when d = 0).
+struct NvScale {
+  uint32_t code;
+  float dec;   // decoded E4M3 scale
+  float inv;   // 1/d
+  bool zero;   // d == 0: all codes of the block are zero
+};
+__device__ __forceinline__ NvScale nv_scale(float amax, float s_x, float g_x) {
+  NvScale s;
+  s.code = cvt_e4m3(__fmul_rn(amax, g_x));
+  s.dec = e4m3_to_f32(s.code);
+  const float d = __fmul_rn(s.dec, s_x);
+  s.zero = d == 0.f;
+  s.inv = s.zero ? 0.f : __frcp_rn(d);
+  return s;
+}
+
+// MXFP4: E8M0 exponent e; multiplier 2^(127-e) (exact); decoded scale 2^(e-127).
+struct MxScale {
+  uint32_t code;
+  float mult, dec;
+  bool zero;
+};
+__device__ __forceinline__ MxScale mx_scale(float amax) {
+  MxScale s;
+  s.zero = amax == 0.f;
+  const int ef = (int)(__float_as_uint(amax) >> 23);
+  s.code = s.zero ? 0u : (uint32_t)max(ef - 2, 0);
+  s.mult = __uint_as_float((254u - s.code) << 23);
+  s.dec = e8m0_to_f32(s.code);
+  return s;
+}
+
+// Codes of 16 values with a multiplier -> 8 bytes in two words (lower K in the low nibble).
+__device__ __forceinline__ void codes16(const float *v, float mult, uint32_t &w0, uint32_t &w1) {
+  float t[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) t[i] = v[i];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mul2(t[2 * i], t[2 * i + 1], mult, mult);
+  uint32_t b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) b[i] = cvt_e2m1x2(t[2 * i], t[2 * i + 1]);
+  w0 = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+  w1 = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+}
+
+// Dequantized values of 4 code bytes (8 values): NVFP4 fp32(fp32(q*dec)*s_x); MXFP4 q*dec.
+template <int FMT>
+__device__ __forceinline__ void deq8(uint32_t w, float dec, float s_x, float *o) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 q = half2_bits_to_float2(cvt_e2m1x2_to_f16x2((w >> (8 * j)) & 0xFFu));
+    o[2 * j] = q.x;
+    o[2 * j + 1] = q.y;
+    mul2(o[2 * j], o[2 * j + 1], dec, dec);  // exact: E2M1 x E4M3 / power of two
+    if (FMT == kFmtNV) mul2(o[2 * j], o[2 * j + 1], s_x, s_x);
+  }
+}
+
+// ---------------------------------------------------------------- one double piece
+// 16 normalized values of double piece `dp` (lane-aligned: dp % 32 == lane).
 template <int FMT, int UNIT, bool DENSE>
-__device__ __forceinline__ void process_chunk(const PrepParams &p, float *v, int row, int c, float s_x,
-                                              float g_x) {
-  uint32_t rb[32];  // residual code bytes (64 codes)
+__device__ __forceinline__ void process16(const PrepParams &p, float *v, int row, int dp, bool live, float s_x,
+                                          float g_x) {
+  const int lane = threadIdx.x & 31;
   if (!DENSE) {
-    // ---- mask: 32 stored values and their metadata
-    float sv[32];
-    uint32_t nib[16];
+    // ---- mask
+    uint32_t nib[4];
+    float gmax = 0.f;
     if (UNIT == 2) {
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
+      for (int g = 0; g < 2; ++g) {
         const float *e = v + 8 * g;
         const float k0 = fmaxf(fabsf(e[0]), fabsf(e[1])), k1 = fmaxf(fabsf(e[2]), fabsf(e[3]));
         const float k2 = fmaxf(fabsf(e[4]), fabsf(e[5])), k3 = fmaxf(fabsf(e[6]), fabsf(e[7]));
-        const uint32_t n = top2_of_4(k0, k1, k2, k3);
-        const uint32_t i0 = n & 3u, i1 = n >> 2;
-        nib[g] = n;
-        sv[4 * g + 0] = sel4(i0, e[0], e[2], e[4], e[6]);
-        sv[4 * g + 1] = sel4(i0, e[1], e[3], e[5], e[7]);
-        sv[4 * g + 2] = sel4(i1, e[0], e[2], e[4], e[6]);
-        sv[4 * g + 3] = sel4(i1, e[1], e[3], e[5], e[7]);
+        nib[g] = top2_of_4(k0, k1, k2, k3);
+        gmax = fmaxf(gmax, fmaxf(fmaxf(k0, k1), fmaxf(k2, k3)));
       }
     } else {
 #pragma unroll
-      for (int g = 0; g < 16; ++g) {
+      for (int g = 0; g < 4; ++g) {
         const float *e = v + 4 * g;
-        const uint32_t n = top2_of_4(fabsf(e[0]), fabsf(e[1]), fabsf(e[2]), fabsf(e[3]));
-        nib[g] = n;
-        sv[2 * g + 0] = sel4(n & 3u, e[0], e[1], e[2], e[3]);
-        sv[2 * g + 1] = sel4(n >> 2, e[0], e[1], e[2], e[3]);
+        const float k0 = fabsf(e[0]), k1 = fabsf(e[1]), k2 = fabsf(e[2]), k3 = fabsf(e[3]);
+        nib[g] = top2_of_4(k0, k1, k2, k3);
+        gmax = fmaxf(gmax, fmaxf(fmaxf(k0, k1), fmaxf(k2, k3)));
       }
     }
-    // ---- backbone quantization (32 stored values)
-    uint32_t sb[16];
-    float dq[32];
-    uint32_t sc_sp;
+    // ---- backbone block amax: 16 stored (NVFP4) = 2 lanes, 32 stored (MXFP4) = 4 lanes
+    gmax = fmaxf(gmax, __shfl_xor_sync(kFull, gmax, 1));
+    if (FMT == kFmtMX) gmax = fmaxf(gmax, __shfl_xor_sync(kFull, gmax, 2));
+    uint32_t sc_code;
+    float mult, dec;
+    bool zero;
     if (FMT == kFmtNV) {
-      const uint32_t s0 = quant_nv<16, true>(sv, s_x, g_x, sb, dq);
-      const uint32_t s1 = quant_nv<16, true>(sv + 16, s_x, g_x, sb + 8, dq + 16);
-      sc_sp = s0 | (s1 << 8);
+      const NvScale s = nv_scale(gmax, s_x, g_x);
+      sc_code = s.code; mult = s.inv; dec = s.dec; zero = s.zero;
     } else {
-      sc_sp = quant_mx<32, true>(sv, sb, dq);
+      const MxScale s = mx_scale(gmax);
+      sc_code = s.code; mult = s.mult; dec = s.dec; zero = s.zero;
     }
-    // ---- residual against the quantized backbone: r = xh - deq at kept positions
+    // ---- backbone codes of all 16 values; keep the selected ones
+    uint32_t w0, w1;
+    codes16(v, mult, w0, w1);
+    if (zero) { w0 = 0u; w1 = 0u; }
+    uint32_t kept, meta;
     if (UNIT == 2) {
-#pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        const uint32_t i0 = nib[g] & 3u, i1 = nib[g] >> 2;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float d0 = (i0 == (uint32_t)j) ? dq[4 * g + 0] : ((i1 == (uint32_t)j) ? dq[4 * g + 2] : 0.f);
-          const float d1 = (i0 == (uint32_t)j) ? dq[4 * g + 1] : ((i1 == (uint32_t)j) ? dq[4 * g + 3] : 0.f);
-          v[8 * g + 2 * j] = __fsub_rn(v[8 * g + 2 * j], d0);
-          v[8 * g + 2 * j + 1] = __fsub_rn(v[8 * g + 2 * j + 1], d1);
-        }
-      }
+      // group g = word g: byte j = pair j; kept bytes i0, i1
+      const uint32_t n0 = nib[0], n1 = nib[1];
+      const uint32_t k0 = __byte_perm(w0, 0u, (n0 & 3u) | ((n0 >> 2) << 4));
+      const uint32_t k1 = __byte_perm(w1, 0u, (n1 & 3u) | ((n1 >> 2) << 4));
+      kept = (k0 & 0xFFFFu) | (k1 << 16);
+      w0 &= (0xFFu << (8 * (n0 & 3u))) | (0xFFu << (8 * (n0 >> 2)));
+      w1 &= (0xFFu << (8 * (n1 & 3u))) | (0xFFu << (8 * (n1 >> 2)));
+      meta = n0 | (n1 << 4);
     } else {
+      // group g = 16 bits (4 nibbles) of the words; kept nibbles i0, i1 -> one byte
+      kept = 0u;
+      meta = 0u;
 #pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        const uint32_t i0 = nib[g] & 3u, i1 = nib[g] >> 2;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float d = (i0 == (uint32_t)j) ? dq[2 * g] : ((i1 == (uint32_t)j) ? dq[2 * g + 1] : 0.f);
-          v[4 * g + j] = __fsub_rn(v[4 * g + j], d);
-        }
+      for (int g = 0; g < 4; ++g) {
+        uint32_t &w = g < 2 ? w0 : w1;
+        const int sh = 16 * (g & 1);
+        const uint32_t n = nib[g], i0 = n & 3u, i1 = n >> 2;
+        const uint32_t q = w >> sh;
+        kept |= (((q >> (4 * i0)) & 0xFu) | (((q >> (4 * i1)) & 0xFu) << 4)) << (8 * g);
+        w &= ~(0xFFFFu << sh) | (((0xFu << (4 * i0)) | (0xFu << (4 * i1))) << sh);
+        meta |= n << (4 * g);
       }
     }
-    // ---- store backbone codes, metadata and scales
-    uint4 *spc = reinterpret_cast<uint4 *>(p.sp_codes + (size_t)row * (p.K / 4) + (size_t)c * 16);
-    *spc = make_uint4(pack4(sb), pack4(sb + 4), pack4(sb + 8), pack4(sb + 12));
-    if (UNIT == 2) {
-      uint32_t m = 0;
+    // ---- residual against the dequantized backbone (dropped codes were zeroed: +0)
+    float dq[16];
+    deq8<FMT>(w0, dec, s_x, dq);
+    deq8<FMT>(w1, dec, s_x, dq + 8);
 #pragma unroll
-      for (int g = 0; g < 8; ++g) m |= nib[g] << (4 * g);
-      uint32_t *dst = reinterpret_cast<uint32_t *>(p.meta + ((size_t)(c >> 2) * p.T_pad + row) * 16 + (c & 3) * 4);
-      *dst = m;
-    } else {
-      uint32_t m0 = 0, m1 = 0;
-#pragma unroll
-      for (int g = 0; g < 8; ++g) { m0 |= nib[g] << (4 * g); m1 |= nib[g + 8] << (4 * g); }
-      uint2 *dst = reinterpret_cast<uint2 *>(p.meta + ((size_t)(c >> 1) * p.T_pad + row) * 16 + (c & 1) * 8);
-      *dst = make_uint2(m0, m1);
+    for (int i = 0; i < 8; ++i) sub2(v[2 * i], v[2 * i + 1], dq[2 * i], dq[2 * i + 1]);
+    // ---- stores: backbone codes (4 bytes per lane), metadata, backbone scales
+    if (live) *reinterpret_cast<uint32_t *>(p.sp_codes + (size_t)row * (p.K / 4) + (size_t)dp * 4) = kept;
+    if (UNIT == 2) {  // 8 bits per lane, 16 lanes per 128-bit slab row
+      const uint32_t m4 = gather4(meta, 1);
+      if (live && (lane & 3) == 0)
+        *reinterpret_cast<uint32_t *>(p.meta + ((size_t)(dp >> 4) * p.T_pad + row) * 16 + ((dp & 15) >> 2) * 4) = m4;
+    } else {  // 16 bits per lane, 8 lanes per slab row
+      const uint32_t m2 = (meta & 0xFFFFu) | (__shfl_down_sync(kFull, meta, 1) << 16);
+      if (live && (lane & 1) == 0)
+        *reinterpret_cast<uint32_t *>(p.meta + ((size_t)(dp >> 3) * p.T_pad + row) * 16 + ((dp & 7) >> 1) * 4) = m2;
     }
-    if (FMT == kFmtNV) {
-      *reinterpret_cast<uint16_t *>(p.sp_scales + atom_offset(row, 2 * c, p.n_sf_sp)) = (uint16_t)sc_sp;
-    } else {
-      p.sp_scales[atom_offset(row, c, p.n_sf_sp)] = (uint8_t)sc_sp;
+    if (FMT == kFmtNV) {  // one scale per 2 lanes: 4 scales from lanes 8q, +2, +4, +6
+      const uint32_t s4 = gather4(sc_code, 2);
+      if (live && (lane & 7) == 0)
+        *reinterpret_cast<uint32_t *>(p.sp_scales + atom_offset(row, dp >> 1, p.n_sf_sp)) = s4;
+    } else {  // one scale per 4 lanes
+      const uint32_t s4 = gather4(sc_code, 4);
+      if (live && (lane & 15) == 0)
+        *reinterpret_cast<uint32_t *>(p.sp_scales + atom_offset(row, dp >> 2, p.n_sf_sp)) = s4;
     }
   }
-  // ---- residual (or, for the dense quantizer, xh itself) in dense blocks
-  uint32_t sc_res;
-  if (FMT == kFmtNV) {
-    uint32_t s[4];
+  // ---- residual (or xh itself for the dense quantizer): dense blocks
+  float am = 0.f;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) s[b] = quant_nv<16, false>(v + 16 * b, s_x, g_x, rb + 8 * b, nullptr);
-    sc_res = s[0] | (s[1] << 8) | (s[2] << 16) | (s[3] << 24);
-    *reinterpret_cast<uint32_t *>(p.res_scales + atom_offset(row, 4 * c, p.n_sf_res)) = sc_res;
-  } else {
-    const uint32_t e0 = quant_mx<32, false>(v, rb, nullptr);
-    const uint32_t e1 = quant_mx<32, false>(v + 32, rb + 16, nullptr);
-    *reinterpret_cast<uint16_t *>(p.res_scales + atom_offset(row, 2 * c, p.n_sf_res)) = (uint16_t)(e0 | (e1 << 8));
+  for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(v[i]));
+  uint32_t r0, r1, rcode;
+  if (FMT == kFmtNV) {  // block = this lane's 16 values
+    const NvScale s = nv_scale(am, s_x, g_x);
+    codes16(v, s.inv, r0, r1);
+    if (s.zero) { r0 = 0u; r1 = 0u; }
+    rcode = s.code;
+    const uint32_t s4 = gather4(rcode, 1);
+    if (live && (lane & 3) == 0)
+      *reinterpret_cast<uint32_t *>(p.res_scales + atom_offset(row, dp, p.n_sf_res)) = s4;
+  } else {  // block of 32 = 2 lanes
+    am = fmaxf(am, __shfl_xor_sync(kFull, am, 1));
+    const MxScale s = mx_scale(am);
+    codes16(v, s.mult, r0, r1);
+    if (s.zero) { r0 = 0u; r1 = 0u; }
+    rcode = s.code;
+    const uint32_t s4 = gather4(rcode, 2);
+    if (live && (lane & 7) == 0)
+      *reinterpret_cast<uint32_t *>(p.res_scales + atom_offset(row, dp >> 1, p.n_sf_res)) = s4;
   }
-  uint4 *rc = reinterpret_cast<uint4 *>(p.res_codes + (size_t)row * (p.K / 2) + (size_t)c * 32);
-  rc[0] = make_uint4(pack4(rb), pack4(rb + 4), pack4(rb + 8), pack4(rb + 12));
-  rc[1] = make_uint4(pack4(rb + 16), pack4(rb + 20), pack4(rb + 24), pack4(rb + 28));
+  if (live) *reinterpret_cast<uint2 *>(p.res_codes + (size_t)row * (p.K / 2) + (size_t)dp * 8) = make_uint2(r0, r1);
 }
 
-// Zero scale / metadata bytes of chunk c for a padding row (rows T..T_pad-1), so the
-// GEMM reads defined values there.
+// Zero the scale and metadata bytes that double piece dp of a padding row (T..T_pad-1)
+// would carry, with the same lane pattern as process16.
 template <int FMT, int UNIT, bool DENSE>
-__device__ __forceinline__ void zero_pad_chunk(const PrepParams &p, int row, int c) {
+__device__ __forceinline__ void zero_pad16(const PrepParams &p, int row, int dp) {
+  const int lane = threadIdx.x & 31;
   if (!DENSE) {
-    if (UNIT == 2)
-      *reinterpret_cast<uint32_t *>(p.meta + ((size_t)(c >> 2) * p.T_pad + row) * 16 + (c & 3) * 4) = 0u;
-    else
-      *reinterpret_cast<uint2 *>(p.meta + ((size_t)(c >> 1) * p.T_pad + row) * 16 + (c & 1) * 8) = make_uint2(0u, 0u);
-    if (FMT == kFmtNV) *reinterpret_cast<uint16_t *>(p.sp_scales + atom_offset(row, 2 * c, p.n_sf_sp)) = 0;
-    else p.sp_scales[atom_offset(row, c, p.n_sf_sp)] = 0;
+    if (UNIT == 2) {
+      if ((lane & 3) == 0)
+        *reinterpret_cast<uint32_t *>(p.meta + ((size_t)(dp >> 4) * p.T_pad + row) * 16 + ((dp & 15) >> 2) * 4) = 0u;
+    } else if ((lane & 1) == 0) {
+      *reinterpret_cast<uint32_t *>(p.meta + ((size_t)(dp >> 3) * p.T_pad + row) * 16 + ((dp & 7) >> 1) * 4) = 0u;
+    }
+    if (FMT == kFmtNV) {
+      if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(p.sp_scales + atom_offset(row, dp >> 1, p.n_sf_sp)) = 0u;
+    } else if ((lane & 15) == 0) {
+      *reinterpret_cast<uint32_t *>(p.sp_scales + atom_offset(row, dp >> 2, p.n_sf_sp)) = 0u;
+    }
   }
-  if (FMT == kFmtNV) *reinterpret_cast<uint32_t *>(p.res_scales + atom_offset(row, 4 * c, p.n_sf_res)) = 0u;
-  else *reinterpret_cast<uint16_t *>(p.res_scales + atom_offset(row, 2 * c, p.n_sf_res)) = 0;
+  if (FMT == kFmtNV) {
+    if ((lane & 3) == 0) *reinterpret_cast<uint32_t *>(p.res_scales + atom_offset(row, dp, p.n_sf_res)) = 0u;
+  } else if ((lane & 7) == 0) {
+    *reinterpret_cast<uint32_t *>(p.res_scales + atom_offset(row, dp >> 1, p.n_sf_res)) = 0u;
+  }
+}
+
+// ---------------------------------------------------------------- team reductions
+// Butterfly within the warp (every lane ends with the identical value), then the W warps of
+// a team combine their partials in a fixed order through shared memory.
+__device__ __forceinline__ double team_sum(double v, int W, int team, int wt, double *sm) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  if (W > 1) {
+    if ((threadIdx.x & 31) == 0) sm[team * 8 + wt] = v;
+    __syncthreads();
+    v = sm[team * 8];
+    for (int i = 1; i < W; ++i) v += sm[team * 8 + i];
+    __syncthreads();
+  }
+  return v;
+}
+
+__device__ __forceinline__ float team_max(float v, int W, int team, int wt, float *sm) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+  if (W > 1) {
+    if ((threadIdx.x & 31) == 0) sm[team * 8 + wt] = v;
+    __syncthreads();
+    v = sm[team * 8];
+    for (int i = 1; i < W; ++i) v = fmaxf(v, sm[team * 8 + i]);
+    __syncthreads();
+  }
+  return v;
 }
 
 __device__ __forceinline__ void row_scales(int fmt, float amax, float &s_x, float &g_x) {
@@ -240,105 +337,93 @@ __device__ __forceinline__ void row_scales(int fmt, float amax, float &s_x, floa
   g_x = __fdiv_rn(448.f, amax);   // = 1 / (6 s_x)
 }
 
-__device__ __forceinline__ float rstd_from(double ss, int K, float eps) {
-  const float ms = __double2float_rn(__ddiv_rn(ss, (double)K));
-  return __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(ms, eps)));
-}
-
-// ---------------------------------------------------------------- kernels
-// Every thread owns at most one 64-element chunk (K <= 64*256) and keeps it in registers.
+// ---------------------------------------------------------------- kernel
 template <int FMT, int UNIT, bool NORM, bool DENSE>
 __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
-  __shared__ double sm_d[8];
-  __shared__ float sm_f[8];
-  const int TS = p.TS;
-  const int team = threadIdx.x / TS;
-  const int c = threadIdx.x - team * TS;
-  const int row = blockIdx.x * (blockDim.x / TS) + team;
-  const bool live = row < p.T && c < p.C;
+  __shared__ double sm_d[64];
+  __shared__ float sm_f[64];
+  const int W = p.TS;                 // warps per row team
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int team = warp / W, wt = warp - team * W;
+  const int row = blockIdx.x * ((blockDim.x >> 5) / W) + team;
+  const int ndp_row = p.K >> 4;       // double pieces per row
+  const int stride = 32 * W;
+  const bool live_row = row < p.T;
 
-  float v[64];
-  if (live) load_bf16x64(p.x + (size_t)row * p.K + (size_t)c * 64, v);
-  else {
+  uint32_t xr[kMaxDP][8];
 #pragma unroll
-    for (int i = 0; i < 64; ++i) v[i] = 0.f;
+  for (int i = 0; i < kMaxDP; ++i) {
+    const int dp = i * stride + wt * 32 + lane;
+    if (live_row && dp < ndp_row) ld256(p.x + (size_t)row * p.K + (size_t)dp * 16, xr[i]);
   }
-  if (NORM) {
-    double ss = 0.0;
-#pragma unroll
-    for (int i = 0; i < 64; ++i) ss = __fma_rn((double)v[i], (double)v[i], ss);
-    ss = team_sum<double>(ss, TS, sm_d);
-    const float rstd = rstd_from(ss, p.K, p.eps);
-    if (live) apply_norm(v, p.gamma + (size_t)c * 64, rstd);
-  }
-  float am = 0.f;
-#pragma unroll
-  for (int i = 0; i < 64; ++i) am = fmaxf(am, fabsf(v[i]));
-  am = team_max(am, TS, sm_f);
-  float s_x, g_x;
-  row_scales(FMT, am, s_x, g_x);
-  if (live) {
-    process_chunk<FMT, UNIT, DENSE>(p, v, row, c, s_x, g_x);
-    if (c == 0) p.row_scale[row] = s_x;
-  } else if (row >= p.T && row < p.T_pad && c < p.C) {
-    zero_pad_chunk<FMT, UNIT, DENSE>(p, row, c);
-  }
-}
 
-// Rows longer than 256 chunks: 256 threads per row, chunks strided by 256, and the
-// input re-read (from L2) in each of the three passes instead of held in registers.
-template <int FMT, int UNIT, bool NORM, bool DENSE>
-__global__ void __launch_bounds__(256) prep_kernel_long(PrepParams p) {
-  __shared__ double sm_d[8];
-  __shared__ float sm_f[8];
-  const int row = blockIdx.x;
-  const int TS = 256;
-  float v[64];
   float rstd = 1.f;
-  if (row >= p.T) {
-    if (row < p.T_pad)
-      for (int c = threadIdx.x; c < p.C; c += TS) zero_pad_chunk<FMT, UNIT, DENSE>(p, row, c);
-    return;
-  }
-  const uint16_t *xr = p.x + (size_t)row * p.K;
   if (NORM) {
     double ss = 0.0;
-    for (int c = threadIdx.x; c < p.C; c += TS) {
-      load_bf16x64(xr + (size_t)c * 64, v);
 #pragma unroll
-      for (int i = 0; i < 64; ++i) ss = __fma_rn((double)v[i], (double)v[i], ss);
+    for (int i = 0; i < kMaxDP; ++i) {
+      const int dp = i * stride + wt * 32 + lane;
+      if (live_row && dp < ndp_row) {
+        float v[16];
+        unpack16(xr[i], v);
+        // float64 per element: bf16 squares are exact and the sum keeps ~2^-53 relative
+        // accuracy, so fp32(sum/K) does not depend on the summation order in practice
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ss = __fma_rn((double)v[j], (double)v[j], ss);
+      }
     }
-    ss = team_sum<double>(ss, TS, sm_d);
-    rstd = rstd_from(ss, p.K, p.eps);
+    ss = team_sum(ss, W, team, wt, sm_d);
+    const float ms = __double2float_rn(__ddiv_rn(ss, (double)p.K));
+    rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, p.eps)));
   }
+
   float am = 0.f;
-  for (int c = threadIdx.x; c < p.C; c += TS) {
-    load_bf16x64(xr + (size_t)c * 64, v);
-    if (NORM) apply_norm(v, p.gamma + (size_t)c * 64, rstd);
 #pragma unroll
-    for (int i = 0; i < 64; ++i) am = fmaxf(am, fabsf(v[i]));
+  for (int i = 0; i < kMaxDP; ++i) {
+    const int dp = i * stride + wt * 32 + lane;
+    if (live_row && dp < ndp_row) {
+      float v[16];
+      unpack16(xr[i], v);
+      if (NORM) normalize16(v, p.gamma + (size_t)dp * 16, rstd);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) am = fmaxf(am, fabsf(v[j]));
+    }
   }
-  am = team_max(am, TS, sm_f);
+  am = team_max(am, W, team, wt, sm_f);
   float s_x, g_x;
   row_scales(FMT, am, s_x, g_x);
-  for (int c = threadIdx.x; c < p.C; c += TS) {
-    load_bf16x64(xr + (size_t)c * 64, v);
-    if (NORM) apply_norm(v, p.gamma + (size_t)c * 64, rstd);
-    process_chunk<FMT, UNIT, DENSE>(p, v, row, c, s_x, g_x);
+
+  const bool pad_row = !live_row && row < p.T_pad;
+#pragma unroll
+  for (int i = 0; i < kMaxDP; ++i) {
+    const int base = i * stride + wt * 32;  // warp-uniform
+    if (base >= ndp_row) break;
+    const int dp = base + lane;
+    const bool live = live_row && dp < ndp_row;
+    if (live_row) {
+      float v[16];
+      if (live) {
+        unpack16(xr[i], v);
+        if (NORM) normalize16(v, p.gamma + (size_t)dp * 16, rstd);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = 0.f;
+      }
+      process16<FMT, UNIT, DENSE>(p, v, row, dp, live, s_x, g_x);
+    } else if (pad_row && dp < ndp_row) {
+      zero_pad16<FMT, UNIT, DENSE>(p, row, dp);
+    }
   }
-  if (threadIdx.x == 0) p.row_scale[row] = s_x;
+  if (live_row && wt == 0 && lane == 0) p.row_scale[row] = s_x;
 }
 
 template <int FMT, int UNIT, bool NORM, bool DENSE>
 cudaError_t launch_t(const PrepParams &p, cudaStream_t st) {
-  if (p.C > 256) {
-    prep_kernel_long<FMT, UNIT, NORM, DENSE><<<p.T_pad, 256, 0, st>>>(p);
-  } else {
-    const int block = p.TS <= 32 ? 256 : p.TS;
-    const int rows_per_block = block / p.TS;
-    const int grid = (p.T_pad + rows_per_block - 1) / rows_per_block;
-    prep_kernel<FMT, UNIT, NORM, DENSE><<<grid, block, 0, st>>>(p);
-  }
+  const int W = p.TS;
+  const int teams = W >= 8 ? 1 : 8 / W;
+  const int block = teams * W * 32;
+  const int grid = (p.T_pad + teams - 1) / teams;
+  prep_kernel<FMT, UNIT, NORM, DENSE><<<grid, block, 0, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -349,21 +434,13 @@ cudaError_t launch_n(const PrepParams &p, bool norm, cudaStream_t st) {
 
 }  // namespace
 
-// Team size: chunks per row rounded up to a power of two within a warp, or to whole
-// warps beyond; rows with more than 256 chunks use the 256-thread strided kernel.
-int prep_team_size(int chunks) {
-  if (chunks > 256) return 256;
-  if (chunks <= 32) {
-    int t = 1;
-    while (t < chunks) t <<= 1;
-    return t;
-  }
-  return (chunks + 31) / 32 * 32;
-}
+// Warps per row: each lane holds at most kMaxDP double pieces (16 elements each).
+int prep_team_warps(int k) { return (k / 16 + 32 * kMaxDP - 1) / (32 * kMaxDP); }
 
 cudaError_t launch_prep(PrepParams p, int fmt, int unit, bool norm, bool dense, cudaStream_t st) {
-  p.C = p.K / 64;
-  p.TS = prep_team_size(p.C);
+  p.C = p.K / 16;
+  p.TS = prep_team_warps(p.K);
+  if (p.TS > 8) return cudaErrorInvalidValue;  // k > 32768: outside the supported range
   if (dense) {
     return fmt == kFmtNV ? launch_n<kFmtNV, 2, true>(p, norm, st) : launch_n<kFmtMX, 2, true>(p, norm, st);
   }

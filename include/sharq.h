@@ -23,7 +23,8 @@
  *    SHARQ_OK or an error status and launches nothing on error; the message is
  *    available from sharq_last_error() (per host thread). No exception crosses
  *    the ABI. A launch failure reported by the CUDA runtime returns SHARQ_ERR_CUDA.
- *  - Device pointers must be 16-byte aligned. bf16 values are raw 16-bit words.
+ *  - Device pointers must be 16-byte aligned (the activation and RMSNorm weight given to
+ *    sharq_prepare / sharq_quantize_dense: 32-byte aligned). bf16 values are raw 16-bit words.
  *  - Sizes: tokens >= 1; k a positive multiple of 256; n_out a positive multiple of 16.
  *
  * Formats. E2M1 element codes (2 per byte, the lower K index in the low nibble)
@@ -41,7 +42,7 @@
  * element pattern (2, 4, 1).
  *
  * Scale layout ("128x4 atoms"). A scale tensor of R rows (R padded to a
- * multiple of 128) and S scales per row (S a multiple of 4) is stored as atoms
+ * multiple of 128; 256 for activations) and S scales per row (S a multiple of 4) is stored as atoms
  * of 512 bytes: atom (R/128 block rb, scale group sg = s/4) at byte offset
  * (rb * S/4 + sg) * 512, and inside it the scale of row r, index s at
  * (r%32)*16 + ((r%128)/32)*4 + s%4. This is the layout the tensor core's
@@ -80,7 +81,7 @@ typedef enum {
  *   resid_codes   [tokens][k/2] bytes: the residual, E2M1 pairs
  *   resid_scales  128x4 atoms, tokens_pad rows, k/B scales per row
  *   row_scale     [tokens] float32: NVFP4 second-level scale s_x (1.0 for MXFP4)
- * tokens_pad = tokens rounded up to 128. */
+ * tokens_pad = tokens rounded up to 256 (the GEMM's CTA pairs cover 256 rows). */
 typedef struct {
   void *sparse_codes;
   void *sparse_meta;

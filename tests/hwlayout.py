@@ -35,7 +35,7 @@ def unswizzle_scales(buf: np.ndarray, rows: int, spr: int) -> np.ndarray:
 
 def meta_to_idx(buf: np.ndarray, tokens: int, k: int, unit: int) -> np.ndarray:
     """Kept unit indices [tokens, G, 2] from metadata slabs (groups of 4 units)."""
-    tp = (tokens + 127) // 128 * 128
+    tp = (tokens + 255) // 256 * 256
     G = k // (4 * unit)
     b = np.asarray(buf, dtype=np.uint8).reshape(-1)
     g = np.arange(G)

@@ -38,9 +38,9 @@ def test_version(S):
 
 
 def test_prep_buffer_sizes(S):
-    T, K = 200, 4096
+    T, K = 300, 4096
     s = S.sharq_prep_buffer_sizes(T, K, 2, 4, 2, "nvfp4")
-    Tp = 256
+    Tp = 512
     assert s == [T * K // 4, (K // 256) * Tp * 16, Tp * K // 32, T * K // 2, Tp * K // 16, T * 4]
     s = S.sharq_prep_buffer_sizes(T, K, 2, 4, 1, "mxfp4")
     assert s == [T * K // 4, (K // 128) * Tp * 16, Tp * K // 64, T * K // 2, Tp * K // 32, T * 4]

@@ -1,9 +1,9 @@
 """Parity of the fused preparation kernel and the dense quantizer with the CPU oracle.
 
 Without RMSNorm (the normalized input held fixed) metadata, codes and scales must be
-bit-exact. With fused RMSNorm the GPU's float64 sum of squares runs in a different order
-from the oracle's, so a row's rstd may differ by one float32 ulp: at most 1e-4 of the
-codes may then differ, each by one E2M1 step.
+bit-exact. With fused RMSNorm the GPU sums the squares in float64 in a different order from the
+oracle, so a row's rstd may (rarely) differ by one float32 ulp: at most 1e-4 of the codes
+may then differ, each by one E2M1 step.
 """
 import numpy as np
 import pytest
@@ -130,18 +130,20 @@ def test_dense_quantizer_matches_oracle(fmt):
     assert np.array_equal(hw.to_np(q.row_scale), ref["row_scale"])
 
 
-@pytest.mark.parametrize("which,T", [("qkv", 2048), ("down", 4096)])
+@pytest.mark.parametrize("which,T", [("qkv", 2048), ("down", 4096), ("qwen_down", 300), ("qwen_qkv", 130)])
 def test_prep_full_size_sampled_rows(which, T):
-    """Full-size workloads in the benchmark's launch configuration; rows are independent, so
-    the oracle checks a sample of them one by one."""
+    """Full-size workloads in the benchmark's launch configuration (and the widest K, 18944,
+    which spreads a row over five warps); rows are independent, so the oracle checks a sample
+    of them one by one."""
     S = require_gpu()
-    lin = wl.llama_qkv(T=T) if which == "qkv" else wl.llama_down(T=T)
+    lin = {"qkv": lambda: wl.llama_qkv(T=T), "down": lambda: wl.llama_down(T=T),
+           "qwen_down": lambda: wl.qwen("down", T), "qwen_qkv": lambda: wl.qwen("qkv", T)}[which]()
     x = to_dev_bf16(lin.x)
     g = to_dev_bf16(lin.gamma) if lin.gamma is not None else None
     p = S.sharq_prepare(x, g, lin.eps, 2, 4, 2, 0)
     torch.cuda.synchronize()
     got = hw.read_prep(p, 16)
-    rows = np.random.default_rng(0).choice(T, 48, replace=False)
+    rows = np.random.default_rng(0).choice(T, min(T, 48), replace=False)
     rows = np.concatenate([rows, [0, T - 1]])
     ref = O.prepare(f32(lin.x[rows]), f32(lin.gamma), lin.eps, 2, 4, 2, O.NVFP4)
     sub = {k: v[rows] for k, v in got.items()}
