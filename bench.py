@@ -273,29 +273,50 @@ def run_sharq(args, rank, world, local):
     t_dl = timeit(lambda: S.sharq_linear_dense(q, wps[0], y=yd, stream=stream))
     del w_bf16
 
-    # ---- end to end through the public API with host buffers (H2D x, D2H y inside the timing)
-    x_host = torch.from_numpy(np.ascontiguousarray(lin.x).view(np.int16)).view(torch.bfloat16).pin_memory()
-    y_host = torch.empty(T, N, dtype=torch.bfloat16).pin_memory()
+    # ---- end to end through the public API with host buffers: every step copies its input
+    # from pinned host memory and its output back. Copies run on their own streams and overlap
+    # the previous/next step's kernels (double-buffered device and host buffers).
+    nb = 2
+    x_host = [torch.from_numpy(np.ascontiguousarray(lin.x).view(np.int16)).view(torch.bfloat16).pin_memory()
+              for _ in range(nb)]
+    y_host = [torch.empty(T, N, dtype=torch.bfloat16).pin_memory() for _ in range(nb)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(nb)]
+    ev_done = [torch.cuda.Event() for _ in range(nb)]
+    ev_out = [torch.cuda.Event() for _ in range(nb)]
 
     def e2e_step(i):
-        s = i % nsets
-        xs[s].copy_(x_host, non_blocking=True)
-        S.sharq_prepare(xs[s], gamma, lin.eps, 2, 4, 2, "nvfp4", out=preps[s], stream=stream)
-        S.sharq_linear(preps[s], wps[s], y=ys[s], stream=stream)
-        y_host.copy_(ys[s], non_blocking=True)
+        b = i % nb
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_done[b])          # buffer b's previous compute finished reading x
+            xs[b].copy_(x_host[b], non_blocking=True)
+            ev_in[b].record(s_in)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])             # buffer b's previous output has been copied out
+        S.sharq_prepare(xs[b], gamma, lin.eps, 2, 4, 2, "nvfp4", out=preps[b], stream=stream)
+        S.sharq_linear(preps[b], wps[b], y=ys[b], stream=stream)
+        ev_done[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[b])
+            y_host[b].copy_(ys[b], non_blocking=True)
+            ev_out[b].record(s_out)
 
+    for e in ev_done + ev_out:
+        e.record(stream)
     for i in range(args.warmup):
         e2e_step(i)
     torch.cuda.synchronize()
     barrier(world)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for i in range(args.steps):
         e2e_step(i)
-    b.record(stream)
+    for e in ev_out:
+        stream.wait_event(e)
+    b_.record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    ms_e2e = max_over_ranks(a.elapsed_time(b), world)
+    ms_e2e = max_over_ranks(a.elapsed_time(b_), world)
     status = S.sharq_device_status()
 
     if rank != 0:

@@ -51,10 +51,10 @@ class _WPack(ctypes.Structure):
                 ("n_out", ctypes.c_int), ("k", ctypes.c_int), ("fmt", ctypes.c_int)]
 
 
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m fp4_activation_sparse_b200.build`")
-    lib = ctypes.CDLL(LIB_PATH)
+def _load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m fp4_activation_sparse_b200.build`")
+    lib = ctypes.CDLL(path)
     P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     sig = {
         "sharq_prep_buffer_sizes": (S, [I, I, I, I, I, I, ctypes.POINTER(S)]),

@@ -168,15 +168,17 @@ __device__ __forceinline__ void tc_commit_both(uint32_t bar) {
       : "memory");
 }
 
-// Shared-memory matrix descriptor (K-major). layout: 0 none, 2 SW128, 4 SW64.
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t sbo_bytes, uint32_t layout, uint32_t lbo_bytes) {
-  uint64_t d = (uint64_t)((addr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= 1ull << 46;  // descriptor version for sm_100
-  d |= (uint64_t)layout << 61;
-  return d;
+// Shared-memory matrix descriptors (K-major) as templates with the address field zero;
+// layout 0 none, 2 SW128, 4 SW64; bit 46 is the sm_100 descriptor version. dsc() adds the
+// 16-byte-unit address of one operand.
+constexpr uint64_t desc_template(uint32_t sbo_bytes, uint32_t layout, uint32_t lbo_bytes) {
+  return ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) | ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) |
+         (1ull << 46) | ((uint64_t)layout << 61);
 }
+constexpr uint64_t kDescSw128 = desc_template(1024, 2, 16);  // 8-row groups of 128 B
+constexpr uint64_t kDescSw64 = desc_template(512, 4, 16);    // 8-row groups of 64 B
+constexpr uint64_t kDescNone = desc_template(128, 0, 0);     // 8 rows x 16 B core matrices
+__device__ __forceinline__ uint64_t dsc(uint64_t tmpl, uint32_t addr16) { return tmpl | (uint64_t)(addr16 & 0x3FFFu); }
 
 // Instruction descriptor of the block-scaled MMA kinds (mxf4 / mxf4nvf4): E2M1 A and B,
 // K-major, fp32 accumulate, M = 256 (two CTAs), N = 256.
@@ -381,47 +383,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int kt = 0; kt < num_k; ++kt) {
           if (!mbar_wait(full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t st = smem0 + stage * kStageBytes;
+          // descriptors: constant templates plus the operand's shared-memory address >> 4
+          const uint32_t st4 = (smem0 + stage * kStageBytes) >> 4;
           const uint32_t sbuf = tmem + kAccCols + (kt & 1) * kScaleBufCols;
           const uint32_t t_meta = sbuf, t_sfa_sp = sbuf + 4, t_sfa_res = sbuf + 12, t_sfb_sp = sbuf + 28,
                          t_sfb_res = sbuf + 44;
           // scales and metadata: shared memory -> tensor memory (both CTAs)
+#pragma unroll
           for (int a = 0; a < apt_res; ++a) {
-            tc_cp_atom(t_sfa_res + 4 * a, sdesc(st + OFF_SFA_RES + a * 512, 128, 0, 0));
-            for (int i = 0; i < 2; ++i)
-              tc_cp_atom(t_sfb_res + 8 * a + 4 * i, sdesc(st + OFF_SFB_RES + i * 2048 + a * 512, 128, 0, 0));
+            tc_cp_atom(t_sfa_res + 4 * a, dsc(kDescNone, st4 + (OFF_SFA_RES + a * 512) / 16));
+            tc_cp_atom(t_sfb_res + 8 * a, dsc(kDescNone, st4 + (OFF_SFB_RES + a * 512) / 16));
+            tc_cp_atom(t_sfb_res + 8 * a + 4, dsc(kDescNone, st4 + (OFF_SFB_RES + 2048 + a * 512) / 16));
           }
           if (SPARSE) {
-            tc_cp_128x128(t_meta, sdesc(st + OFF_META, 128, 0, 0));
+            tc_cp_128x128(t_meta, dsc(kDescNone, st4 + OFF_META / 16));
+#pragma unroll
             for (int a = 0; a < apt_sp; ++a) {
-              tc_cp_atom(t_sfa_sp + 4 * a, sdesc(st + OFF_SFA_SP + a * 512, 128, 0, 0));
-              for (int i = 0; i < 2; ++i)
-                tc_cp_atom(t_sfb_sp + 8 * a + 4 * i, sdesc(st + OFF_SFB_SP + i * 1024 + a * 512, 128, 0, 0));
+              tc_cp_atom(t_sfa_sp + 4 * a, dsc(kDescNone, st4 + (OFF_SFA_SP + a * 512) / 16));
+              tc_cp_atom(t_sfb_sp + 8 * a, dsc(kDescNone, st4 + (OFF_SFB_SP + a * 512) / 16));
+              tc_cp_atom(t_sfb_sp + 8 * a + 4, dsc(kDescNone, st4 + (OFF_SFB_SP + 1024 + a * 512) / 16));
             }
           }
           uint32_t accumulate = kt > 0 ? 1u : 0u;
           if (SPARSE) {
             // two sparse MMAs: 128 logical K each = 32 bytes of compressed A, 64 bytes of B
+#pragma unroll
             for (int j = 0; j < 2; ++j) {
-              const uint64_t ad = sdesc(st + OFF_ASP + 32 * j, 512, 4, 16);
-              const uint64_t bd = sdesc(st + OFF_B + 64 * j, 1024, 2, 16);
               // NVFP4: 4 scales per row per MMA (one atom, id 0); MXFP4: 2 (half an atom)
               const uint32_t atom = MX ? (uint32_t)(j >> 1) : (uint32_t)j;
               const uint32_t id = MX ? (uint32_t)(2 * (j & 1)) : 0u;
-              const uint32_t sfa = (t_sfa_sp + 4 * atom) | (id << 30);
-              const uint32_t sfb = (t_sfb_sp + 8 * atom) | (id << 30);
-              mma_sparse<MX>(acc, ad, bd, t_meta + 2 * j, idesc_bs(true, MX, id, id), sfa, sfb, accumulate);
+              mma_sparse<MX>(acc, dsc(kDescSw64, st4 + (OFF_ASP + 32 * j) / 16),
+                             dsc(kDescSw128, st4 + (OFF_B + 64 * j) / 16), t_meta + 2 * j, idesc_bs(true, MX, id, id),
+                             (t_sfa_sp + 4 * atom) | (id << 30), (t_sfb_sp + 8 * atom) | (id << 30), accumulate);
               accumulate = 1u;
             }
           }
+#pragma unroll
           for (int j = 0; j < 4; ++j) {  // four dense MMAs of K = 64 (32 bytes of A and B)
-            const uint64_t ad = sdesc(st + OFF_ARES + 32 * j, 1024, 2, 16);
-            const uint64_t bd = sdesc(st + OFF_B + 32 * j, 1024, 2, 16);
             const uint32_t atom = MX ? (uint32_t)(j >> 1) : (uint32_t)j;
             const uint32_t id = MX ? (uint32_t)(2 * (j & 1)) : 0u;
-            const uint32_t sfa = (t_sfa_res + 4 * atom) | (id << 30);
-            const uint32_t sfb = (t_sfb_res + 8 * atom) | (id << 30);
-            mma_dense<MX>(acc, ad, bd, idesc_bs(false, MX, id, id), sfa, sfb, accumulate);
+            mma_dense<MX>(acc, dsc(kDescSw128, st4 + (OFF_ARES + 32 * j) / 16),
+                          dsc(kDescSw128, st4 + (OFF_B + 32 * j) / 16), idesc_bs(false, MX, id, id),
+                          (t_sfa_res + 4 * atom) | (id << 30), (t_sfb_res + 8 * atom) | (id << 30), accumulate);
             accumulate = 1u;
           }
           tc_commit_both(empty_bar(stage));  // frees the stage in both CTAs once these MMAs have read it

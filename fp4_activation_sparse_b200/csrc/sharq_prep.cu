@@ -9,16 +9,17 @@
 // One read of the bf16 activations. A team of W warps owns one token row (W = K/4096
 // rounded up); every lane owns "double pieces" of 16 consecutive K elements (one 256-bit
 // load), consecutive lanes owning consecutive pieces, and keeps its whole share of the
-// row in registers. Passes over those registers: sum of squares (RMSNorm), row amax
-// (second-level scale), then per double piece:
-//   mask (2 groups of 4 pairs / 4 groups of 4 elements) -> backbone block amax (the
-//   largest element of a group is always kept, so it is the max of group maxima) ->
-//   backbone codes for every element with the backbone block scale; the kept bytes are
-//   stored, the dropped ones zeroed -> dequantized backbone -> residual r = xh - deq ->
-//   residual block scale and codes.
-// Blocks spanning lanes reduce with warp shuffles; scale and metadata bytes are gathered
-// by shuffles into whole 32-bit words, so every store is coalesced. Float32 arithmetic
-// uses explicit round-to-nearest operations, so no contraction changes a rounding.
+// row in registers. Passes over those registers: sum of squares (RMSNorm, float64), row
+// amax (second-level scale), then per double piece:
+//   mask (2 groups of 4 pairs / 4 groups of 4 elements; a tournament picks the two
+//   largest keys) -> backbone block amax (the largest element of a group is always kept,
+//   so it is the max of the group maxima) -> backbone codes for every element with the
+//   backbone block scale; the kept bytes are stored, the dropped ones zeroed ->
+//   dequantized backbone -> residual r = xh - deq -> residual block scale and codes.
+// Blocks spanning lanes reduce with warp shuffles; scales and metadata are written as
+// bytes straight into their 128x4-atom / slab layouts. The RMSNorm weight is staged once
+// per block in shared memory as float32. Float32 arithmetic uses explicit
+// round-to-nearest scalar operations, so no contraction changes a rounding.
 #include "sharq_common.cuh"
 #include "sharq_internal.h"
 
@@ -29,35 +30,19 @@ namespace {
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr int kMaxDP = 8;  // double pieces (16 elements) per lane
 
-// mask of kept units (bit i = unit i kept) -> metadata nibble i0 | i1 << 2
-constexpr unsigned long long kNibbleLut =
-    (4ull << (3 * 4)) | (8ull << (5 * 4)) | (9ull << (6 * 4)) | (12ull << (9 * 4)) |
-    (13ull << (10 * 4)) | (14ull << (12 * 4));
-
-// Top-2 of four keys, ties to the lower index: the two units whose rank
-// (#keys strictly above + #equal keys at a lower index) is below 2.
-__device__ __forceinline__ uint32_t top2_of_4(float k0, float k1, float k2, float k3) {
-  int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
-  if (k0 >= k1) ++r1; else ++r0;
-  if (k0 >= k2) ++r2; else ++r0;
-  if (k0 >= k3) ++r3; else ++r0;
-  if (k1 >= k2) ++r2; else ++r1;
-  if (k1 >= k3) ++r3; else ++r1;
-  if (k2 >= k3) ++r3; else ++r2;
-  const uint32_t m = (r0 < 2) | ((r1 < 2) << 1) | ((r2 < 2) << 2) | ((r3 < 2) << 3);
-  return (uint32_t)(kNibbleLut >> (m * 4)) & 0xFu;
-}
-
-// ---------------------------------------------------------------- float32 pairs
-// Element-wise round-to-nearest products / differences of two lanes. (Scalar operations:
-// the packed f32x2 forms were measured not to round like these on every input.)
-__device__ __forceinline__ void mul2(float &a0, float &a1, float b0, float b1) {
-  a0 = __fmul_rn(a0, b0);
-  a1 = __fmul_rn(a1, b1);
-}
-__device__ __forceinline__ void sub2(float &a0, float &a1, float b0, float b1) {
-  a0 = __fsub_rn(a0, b0);
-  a1 = __fsub_rn(a1, b1);
+// The two largest of four keys, ties to the lower index, as a metadata nibble i0 | i1 << 2
+// (i0 < i1); also returns the largest key. Tournament: winners and losers of (0,1) and
+// (2,3), the overall winner, then the runner-up among the winner's pair loser and the other
+// pair's winner (on equal keys the lower index wins every comparison).
+__device__ __forceinline__ uint32_t top2_of_4(float k0, float k1, float k2, float k3, float &kmax) {
+  const bool c01 = k0 >= k1, c23 = k2 >= k3;
+  const float hi01 = fmaxf(k0, k1), lo01 = fminf(k0, k1), hi23 = fmaxf(k2, k3), lo23 = fminf(k2, k3);
+  const uint32_t ih01 = c01 ? 0u : 1u, il01 = ih01 ^ 1u, ih23 = c23 ? 2u : 3u, il23 = ih23 ^ 1u;
+  const bool cw = hi01 >= hi23;
+  const uint32_t first = cw ? ih01 : ih23;
+  const uint32_t second = cw ? (lo01 >= hi23 ? il01 : ih23) : (hi01 >= lo23 ? ih01 : il23);
+  kmax = fmaxf(hi01, hi23);
+  return min(first, second) | (max(first, second) << 2);
 }
 
 // ---------------------------------------------------------------- I/O
@@ -75,32 +60,34 @@ __device__ __forceinline__ void unpack16(const uint32_t (&w)[8], float *v) {
   }
 }
 
-// xh = fp32(fp32(x * rstd) * gamma) for 16 values
-__device__ __forceinline__ void normalize16(float *v, const uint16_t *gamma16, float rstd) {
-  uint32_t g[8];
-  ld256(gamma16, g);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    mul2(v[2 * i], v[2 * i + 1], rstd, rstd);
-    mul2(v[2 * i], v[2 * i + 1], bf16lo(g[i]), bf16hi(g[i]));
-  }
+// Float offset of element k of the RMSNorm weight in shared memory: [dp / 32][chunk][lane][4]
+// with dp = k / 16, chunk = (k % 16) / 4, so a warp's 32 lanes read 32 consecutive 16-byte
+// chunks (no bank conflicts).
+__device__ __forceinline__ int gamma_smem_index(int k) {
+  const int dp = k >> 4, c = (k >> 2) & 3;
+  return ((((dp >> 5) << 2) + c) * 32 + (dp & 31)) * 4 + (k & 3);
 }
 
-// Gather byte b of lanes (lane, lane+d, lane+2d, lane+3d) into one word (valid on the first).
-__device__ __forceinline__ uint32_t gather4(uint32_t b, int d) {
-  const uint32_t b1 = __shfl_down_sync(kFull, b, d);
-  const uint32_t b2 = __shfl_down_sync(kFull, b, 2 * d);
-  const uint32_t b3 = __shfl_down_sync(kFull, b, 3 * d);
-  return (b & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
+// xh = fp32(fp32(x * rstd) * gamma) for the 16 values of double piece dp
+__device__ __forceinline__ void normalize16(float *v, const float *gs, int dp, float rstd) {
+  const float4 *g4 = reinterpret_cast<const float4 *>(gs);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float4 g = g4[(((dp >> 5) << 2) + c) * 32 + (dp & 31)];
+    v[4 * c + 0] = __fmul_rn(__fmul_rn(v[4 * c + 0], rstd), g.x);
+    v[4 * c + 1] = __fmul_rn(__fmul_rn(v[4 * c + 1], rstd), g.y);
+    v[4 * c + 2] = __fmul_rn(__fmul_rn(v[4 * c + 2], rstd), g.z);
+    v[4 * c + 3] = __fmul_rn(__fmul_rn(v[4 * c + 3], rstd), g.w);
+  }
 }
 
 // ---------------------------------------------------------------- block scales
 // NVFP4: E4M3 code of fp32(amax*g); d = fp32(dec*s); inv = 1/d (0 when d = 0).
 struct NvScale {
   uint32_t code;
-  float dec;   // decoded E4M3 scale
-  float inv;   // 1/d
-  bool zero;   // d == 0: all codes of the block are zero
+  float dec;  // decoded E4M3 scale
+  float inv;  // 1/d
+  bool zero;  // d == 0: all codes of the block are zero
 };
 __device__ __forceinline__ NvScale nv_scale(float amax, float s_x, float g_x) {
   NvScale s;
@@ -128,39 +115,51 @@ __device__ __forceinline__ MxScale mx_scale(float amax) {
   return s;
 }
 
-// Codes of 16 values with a multiplier -> 8 bytes in two words (lower K in the low nibble).
+// Codes of 16 values scaled by `mult` -> two words (lower K in the low nibble).
 __device__ __forceinline__ void codes16(const float *v, float mult, uint32_t &w0, uint32_t &w1) {
   float t[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) t[i] = v[i];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) mul2(t[2 * i], t[2 * i + 1], mult, mult);
-  uint32_t b[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) b[i] = cvt_e2m1x2(t[2 * i], t[2 * i + 1]);
-  w0 = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-  w1 = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+  for (int i = 0; i < 16; ++i) t[i] = __fmul_rn(v[i], mult);
+  w0 = cvt_e2m1x8(t[0], t[1], t[2], t[3], t[4], t[5], t[6], t[7]);
+  w1 = cvt_e2m1x8(t[8], t[9], t[10], t[11], t[12], t[13], t[14], t[15]);
 }
 
-// Dequantized values of 4 code bytes (8 values): NVFP4 fp32(fp32(q*dec)*s_x); MXFP4 q*dec.
+// Dequantized values of one word of codes (8 values): NVFP4 fp32(fp32(q*dec)*s_x) with the
+// exact product q*dec taken in half precision; MXFP4 q*dec (exact).
 template <int FMT>
 __device__ __forceinline__ void deq8(uint32_t w, float dec, float s_x, float *o) {
+  uint32_t h[4];
+  cvt_e2m1x8_to_f16x2(w, h);
+  if (FMT == kFmtNV) {
+    const __half2 d2 = __float2half2_rn(dec);  // E4M3 values are exact in half precision
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float2 q = half2_bits_to_float2(cvt_e2m1x2_to_f16x2((w >> (8 * j)) & 0xFFu));
-    o[2 * j] = q.x;
-    o[2 * j + 1] = q.y;
-    mul2(o[2 * j], o[2 * j + 1], dec, dec);  // exact: E2M1 x E4M3 / power of two
-    if (FMT == kFmtNV) mul2(o[2 * j], o[2 * j + 1], s_x, s_x);
+    for (int j = 0; j < 4; ++j) {
+      const __half2 q = __hmul2(*reinterpret_cast<const __half2 *>(&h[j]), d2);  // exact (<= 6 significant bits)
+      const float2 f = __half22float2(q);
+      o[2 * j] = __fmul_rn(f.x, s_x);
+      o[2 * j + 1] = __fmul_rn(f.y, s_x);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = half2_bits_to_float2(h[j]);
+      o[2 * j] = __fmul_rn(f.x, dec);
+      o[2 * j + 1] = __fmul_rn(f.y, dec);
+    }
   }
 }
+
+// Byte offset of scale s of `row` in a 128x4-atom scale tensor: row part + scale part.
+__device__ __forceinline__ size_t atom_row_part(int row, int spr) {
+  return (size_t)(row >> 7) * (spr >> 2) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4;
+}
+__device__ __forceinline__ size_t atom_scale_part(int s) { return (size_t)(s >> 2) * 512 + (s & 3); }
 
 // ---------------------------------------------------------------- one double piece
 // 16 normalized values of double piece `dp` (lane-aligned: dp % 32 == lane).
 template <int FMT, int UNIT, bool DENSE>
 __device__ __forceinline__ void process16(const PrepParams &p, float *v, int row, int dp, bool live, float s_x,
-                                          float g_x) {
-  const int lane = threadIdx.x & 31;
+                                          float g_x, size_t sp_row, size_t res_row) {
   if (!DENSE) {
     // ---- mask
     uint32_t nib[4];
@@ -169,18 +168,18 @@ __device__ __forceinline__ void process16(const PrepParams &p, float *v, int row
 #pragma unroll
       for (int g = 0; g < 2; ++g) {
         const float *e = v + 8 * g;
-        const float k0 = fmaxf(fabsf(e[0]), fabsf(e[1])), k1 = fmaxf(fabsf(e[2]), fabsf(e[3]));
-        const float k2 = fmaxf(fabsf(e[4]), fabsf(e[5])), k3 = fmaxf(fabsf(e[6]), fabsf(e[7]));
-        nib[g] = top2_of_4(k0, k1, k2, k3);
-        gmax = fmaxf(gmax, fmaxf(fmaxf(k0, k1), fmaxf(k2, k3)));
+        float km;
+        nib[g] = top2_of_4(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3])),
+                           fmaxf(fabsf(e[4]), fabsf(e[5])), fmaxf(fabsf(e[6]), fabsf(e[7])), km);
+        gmax = fmaxf(gmax, km);
       }
     } else {
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         const float *e = v + 4 * g;
-        const float k0 = fabsf(e[0]), k1 = fabsf(e[1]), k2 = fabsf(e[2]), k3 = fabsf(e[3]);
-        nib[g] = top2_of_4(k0, k1, k2, k3);
-        gmax = fmaxf(gmax, fmaxf(fmaxf(k0, k1), fmaxf(k2, k3)));
+        float km;
+        nib[g] = top2_of_4(fabsf(e[0]), fabsf(e[1]), fabsf(e[2]), fabsf(e[3]), km);
+        gmax = fmaxf(gmax, km);
       }
     }
     // ---- backbone block amax: 16 stored (NVFP4) = 2 lanes, 32 stored (MXFP4) = 4 lanes
@@ -206,7 +205,7 @@ __device__ __forceinline__ void process16(const PrepParams &p, float *v, int row
       const uint32_t n0 = nib[0], n1 = nib[1];
       const uint32_t k0 = __byte_perm(w0, 0u, (n0 & 3u) | ((n0 >> 2) << 4));
       const uint32_t k1 = __byte_perm(w1, 0u, (n1 & 3u) | ((n1 >> 2) << 4));
-      kept = (k0 & 0xFFFFu) | (k1 << 16);
+      kept = __byte_perm(k0, k1, 0x5410);
       w0 &= (0xFFu << (8 * (n0 & 3u))) | (0xFFu << (8 * (n0 >> 2)));
       w1 &= (0xFFu << (8 * (n1 & 3u))) | (0xFFu << (8 * (n1 >> 2)));
       meta = n0 | (n1 << 4);
@@ -230,77 +229,57 @@ __device__ __forceinline__ void process16(const PrepParams &p, float *v, int row
     deq8<FMT>(w0, dec, s_x, dq);
     deq8<FMT>(w1, dec, s_x, dq + 8);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) sub2(v[2 * i], v[2 * i + 1], dq[2 * i], dq[2 * i + 1]);
-    // ---- stores: backbone codes (4 bytes per lane), metadata, backbone scales
-    if (live) *reinterpret_cast<uint32_t *>(p.sp_codes + (size_t)row * (p.K / 4) + (size_t)dp * 4) = kept;
-    if (UNIT == 2) {  // 8 bits per lane, 16 lanes per 128-bit slab row
-      const uint32_t m4 = gather4(meta, 1);
-      if (live && (lane & 3) == 0)
-        *reinterpret_cast<uint32_t *>(p.meta + ((size_t)(dp >> 4) * p.T_pad + row) * 16 + ((dp & 15) >> 2) * 4) = m4;
-    } else {  // 16 bits per lane, 8 lanes per slab row
-      const uint32_t m2 = (meta & 0xFFFFu) | (__shfl_down_sync(kFull, meta, 1) << 16);
-      if (live && (lane & 1) == 0)
-        *reinterpret_cast<uint32_t *>(p.meta + ((size_t)(dp >> 3) * p.T_pad + row) * 16 + ((dp & 7) >> 1) * 4) = m2;
-    }
-    if (FMT == kFmtNV) {  // one scale per 2 lanes: 4 scales from lanes 8q, +2, +4, +6
-      const uint32_t s4 = gather4(sc_code, 2);
-      if (live && (lane & 7) == 0)
-        *reinterpret_cast<uint32_t *>(p.sp_scales + atom_offset(row, dp >> 1, p.n_sf_sp)) = s4;
-    } else {  // one scale per 4 lanes
-      const uint32_t s4 = gather4(sc_code, 4);
-      if (live && (lane & 15) == 0)
-        *reinterpret_cast<uint32_t *>(p.sp_scales + atom_offset(row, dp >> 2, p.n_sf_sp)) = s4;
+    for (int i = 0; i < 16; ++i) v[i] = __fsub_rn(v[i], dq[i]);
+    // ---- stores: backbone codes (4 bytes per lane), metadata and backbone scale bytes
+    if (live) {
+      *reinterpret_cast<uint32_t *>(p.sp_codes + (size_t)row * (p.K / 4) + (size_t)dp * 4) = kept;
+      if (UNIT == 2)  // 8 bits per lane, 16 lanes per 128-bit slab row
+        p.meta[((size_t)(dp >> 4) * p.T_pad + row) * 16 + (dp & 15)] = (uint8_t)meta;
+      else  // 16 bits per lane, 8 lanes per slab row
+        *reinterpret_cast<uint16_t *>(p.meta + ((size_t)(dp >> 3) * p.T_pad + row) * 16 + (dp & 7) * 2) =
+            (uint16_t)meta;
+      if (FMT == kFmtNV) {  // one backbone scale per 2 lanes
+        if ((dp & 1) == 0) p.sp_scales[sp_row + atom_scale_part(dp >> 1)] = (uint8_t)sc_code;
+      } else if ((dp & 3) == 0) {  // one per 4 lanes
+        p.sp_scales[sp_row + atom_scale_part(dp >> 2)] = (uint8_t)sc_code;
+      }
     }
   }
   // ---- residual (or xh itself for the dense quantizer): dense blocks
   float am = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(v[i]));
-  uint32_t r0, r1, rcode;
+  uint32_t r0, r1;
   if (FMT == kFmtNV) {  // block = this lane's 16 values
     const NvScale s = nv_scale(am, s_x, g_x);
     codes16(v, s.inv, r0, r1);
     if (s.zero) { r0 = 0u; r1 = 0u; }
-    rcode = s.code;
-    const uint32_t s4 = gather4(rcode, 1);
-    if (live && (lane & 3) == 0)
-      *reinterpret_cast<uint32_t *>(p.res_scales + atom_offset(row, dp, p.n_sf_res)) = s4;
+    if (live) p.res_scales[res_row + atom_scale_part(dp)] = (uint8_t)s.code;
   } else {  // block of 32 = 2 lanes
     am = fmaxf(am, __shfl_xor_sync(kFull, am, 1));
     const MxScale s = mx_scale(am);
     codes16(v, s.mult, r0, r1);
     if (s.zero) { r0 = 0u; r1 = 0u; }
-    rcode = s.code;
-    const uint32_t s4 = gather4(rcode, 2);
-    if (live && (lane & 7) == 0)
-      *reinterpret_cast<uint32_t *>(p.res_scales + atom_offset(row, dp >> 1, p.n_sf_res)) = s4;
+    if (live && (dp & 1) == 0) p.res_scales[res_row + atom_scale_part(dp >> 1)] = (uint8_t)s.code;
   }
   if (live) *reinterpret_cast<uint2 *>(p.res_codes + (size_t)row * (p.K / 2) + (size_t)dp * 8) = make_uint2(r0, r1);
 }
 
 // Zero the scale and metadata bytes that double piece dp of a padding row (T..T_pad-1)
-// would carry, with the same lane pattern as process16.
+// would carry.
 template <int FMT, int UNIT, bool DENSE>
-__device__ __forceinline__ void zero_pad16(const PrepParams &p, int row, int dp) {
-  const int lane = threadIdx.x & 31;
+__device__ __forceinline__ void zero_pad16(const PrepParams &p, int row, int dp, size_t sp_row, size_t res_row) {
   if (!DENSE) {
-    if (UNIT == 2) {
-      if ((lane & 3) == 0)
-        *reinterpret_cast<uint32_t *>(p.meta + ((size_t)(dp >> 4) * p.T_pad + row) * 16 + ((dp & 15) >> 2) * 4) = 0u;
-    } else if ((lane & 1) == 0) {
-      *reinterpret_cast<uint32_t *>(p.meta + ((size_t)(dp >> 3) * p.T_pad + row) * 16 + ((dp & 7) >> 1) * 4) = 0u;
-    }
+    if (UNIT == 2) p.meta[((size_t)(dp >> 4) * p.T_pad + row) * 16 + (dp & 15)] = 0;
+    else *reinterpret_cast<uint16_t *>(p.meta + ((size_t)(dp >> 3) * p.T_pad + row) * 16 + (dp & 7) * 2) = 0;
     if (FMT == kFmtNV) {
-      if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(p.sp_scales + atom_offset(row, dp >> 1, p.n_sf_sp)) = 0u;
-    } else if ((lane & 15) == 0) {
-      *reinterpret_cast<uint32_t *>(p.sp_scales + atom_offset(row, dp >> 2, p.n_sf_sp)) = 0u;
+      if ((dp & 1) == 0) p.sp_scales[sp_row + atom_scale_part(dp >> 1)] = 0;
+    } else if ((dp & 3) == 0) {
+      p.sp_scales[sp_row + atom_scale_part(dp >> 2)] = 0;
     }
   }
-  if (FMT == kFmtNV) {
-    if ((lane & 3) == 0) *reinterpret_cast<uint32_t *>(p.res_scales + atom_offset(row, dp, p.n_sf_res)) = 0u;
-  } else if ((lane & 7) == 0) {
-    *reinterpret_cast<uint32_t *>(p.res_scales + atom_offset(row, dp >> 1, p.n_sf_res)) = 0u;
-  }
+  if (FMT == kFmtNV) p.res_scales[res_row + atom_scale_part(dp)] = 0;
+  else if ((dp & 1) == 0) p.res_scales[res_row + atom_scale_part(dp >> 1)] = 0;
 }
 
 // ---------------------------------------------------------------- team reductions
@@ -340,13 +319,15 @@ __device__ __forceinline__ void row_scales(int fmt, float amax, float &s_x, floa
 // ---------------------------------------------------------------- kernel
 template <int FMT, int UNIT, bool NORM, bool DENSE>
 __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
+  extern __shared__ float4 gamma_smem4[];  // NORM: the RMSNorm weight as float32 (K rounded up to 512)
   __shared__ double sm_d[64];
   __shared__ float sm_f[64];
-  const int W = p.TS;                 // warps per row team
+  float *gs = reinterpret_cast<float *>(gamma_smem4);
+  const int W = p.TS;  // warps per row team
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int team = warp / W, wt = warp - team * W;
   const int row = blockIdx.x * ((blockDim.x >> 5) / W) + team;
-  const int ndp_row = p.K >> 4;       // double pieces per row
+  const int ndp_row = p.K >> 4;  // double pieces per row
   const int stride = 32 * W;
   const bool live_row = row < p.T;
 
@@ -359,6 +340,12 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
 
   float rstd = 1.f;
   if (NORM) {
+    // stage gamma (bf16 -> float32) once per block while the row loads are in flight
+    for (int k = 2 * threadIdx.x; k < p.K; k += 2 * blockDim.x) {
+      const uint32_t g2 = *reinterpret_cast<const uint32_t *>(p.gamma + k);
+      gs[gamma_smem_index(k)] = bf16lo(g2);
+      gs[gamma_smem_index(k + 1)] = bf16hi(g2);
+    }
     double ss = 0.0;
 #pragma unroll
     for (int i = 0; i < kMaxDP; ++i) {
@@ -372,6 +359,7 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
         for (int j = 0; j < 16; ++j) ss = __fma_rn((double)v[j], (double)v[j], ss);
       }
     }
+    __syncthreads();  // gamma staged
     ss = team_sum(ss, W, team, wt, sm_d);
     const float ms = __double2float_rn(__ddiv_rn(ss, (double)p.K));
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, p.eps)));
@@ -384,7 +372,7 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
     if (live_row && dp < ndp_row) {
       float v[16];
       unpack16(xr[i], v);
-      if (NORM) normalize16(v, p.gamma + (size_t)dp * 16, rstd);
+      if (NORM) normalize16(v, gs, dp, rstd);
 #pragma unroll
       for (int j = 0; j < 16; ++j) am = fmaxf(am, fabsf(v[j]));
     }
@@ -393,6 +381,8 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   float s_x, g_x;
   row_scales(FMT, am, s_x, g_x);
 
+  const size_t sp_row = DENSE ? 0 : atom_row_part(row, p.n_sf_sp);
+  const size_t res_row = atom_row_part(row, p.n_sf_res);
   const bool pad_row = !live_row && row < p.T_pad;
 #pragma unroll
   for (int i = 0; i < kMaxDP; ++i) {
@@ -404,14 +394,14 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
       float v[16];
       if (live) {
         unpack16(xr[i], v);
-        if (NORM) normalize16(v, p.gamma + (size_t)dp * 16, rstd);
+        if (NORM) normalize16(v, gs, dp, rstd);
       } else {
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = 0.f;
       }
-      process16<FMT, UNIT, DENSE>(p, v, row, dp, live, s_x, g_x);
+      process16<FMT, UNIT, DENSE>(p, v, row, dp, live, s_x, g_x, sp_row, res_row);
     } else if (pad_row && dp < ndp_row) {
-      zero_pad16<FMT, UNIT, DENSE>(p, row, dp);
+      zero_pad16<FMT, UNIT, DENSE>(p, row, dp, sp_row, res_row);
     }
   }
   if (live_row && wt == 0 && lane == 0) p.row_scale[row] = s_x;
@@ -423,7 +413,14 @@ cudaError_t launch_t(const PrepParams &p, cudaStream_t st) {
   const int teams = W >= 8 ? 1 : 8 / W;
   const int block = teams * W * 32;
   const int grid = (p.T_pad + teams - 1) / teams;
-  prep_kernel<FMT, UNIT, NORM, DENSE><<<grid, block, 0, st>>>(p);
+  // the staging layout reserves 512 floats per 32 double pieces: round K up to 512
+  const size_t smem = NORM ? (size_t)((p.K + 511) / 512 * 512) * sizeof(float) : 0;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(prep_kernel<FMT, UNIT, NORM, DENSE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  prep_kernel<FMT, UNIT, NORM, DENSE><<<grid, block, smem, st>>>(p);
   return cudaGetLastError();
 }
 
