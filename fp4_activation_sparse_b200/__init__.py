@@ -1,8 +1,10 @@
 """Python binding of libsharq: SharQ's online sparse-dense FP4 linear layer on B200.
 
 Argument marshalling only (ctypes). Every computation runs in the library's CUDA
-kernels; torch supplies device memory and streams. There is no CPU fallback: if
-``libsharq.so`` is missing, importing this package raises.
+kernels; torch supplies device memory and streams. There is no CPU fallback: the
+library is loaded on first use (so that ``fp4_activation_sparse_b200.build`` can run on
+a fresh tree), and every call raises ImportError if ``libsharq.so`` is missing or does
+not export what this binding expects.
 
 The three calls of the method ("SharQ: Bridging Activation Sparsity and FP4
 Quantization for LLM Inference", Abstract):
@@ -38,16 +40,13 @@ class SharqError(RuntimeError):
 
 
 class _Prep(ctypes.Structure):
-    _fields_ = [("sparse_codes", ctypes.c_void_p), ("sparse_meta", ctypes.c_void_p),
-                ("sparse_scales", ctypes.c_void_p), ("resid_codes", ctypes.c_void_p),
-                ("resid_scales", ctypes.c_void_p), ("row_scale", ctypes.c_void_p),
+    _fields_ = [("tiles", ctypes.c_void_p), ("row_scale", ctypes.c_void_p),
                 ("tokens", ctypes.c_int), ("k", ctypes.c_int), ("nm_n", ctypes.c_int),
                 ("nm_m", ctypes.c_int), ("unit", ctypes.c_int), ("fmt", ctypes.c_int)]
 
 
 class _WPack(ctypes.Structure):
-    _fields_ = [("codes", ctypes.c_void_p), ("scales_sparse", ctypes.c_void_p),
-                ("scales_dense", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
+    _fields_ = [("tiles", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
                 ("n_out", ctypes.c_int), ("k", ctypes.c_int), ("fmt", ctypes.c_int)]
 
 
@@ -55,15 +54,18 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
         raise ImportError(f"{path} is missing: build it with `python -m fp4_activation_sparse_b200.build`")
     lib = ctypes.CDLL(path)
+    if not hasattr(lib, "sharq_dense_buffer_sizes"):
+        raise ImportError(f"{path} is stale (ABI older than this binding): rebuild it")
     P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     sig = {
         "sharq_prep_buffer_sizes": (S, [I, I, I, I, I, I, ctypes.POINTER(S)]),
+        "sharq_dense_buffer_sizes": (S, [I, I, I, ctypes.POINTER(S)]),
         "sharq_wpack_buffer_sizes": (S, [I, I, I, ctypes.POINTER(S)]),
         "sharq_pack_weight": (I, [P, I, I, I, ctypes.POINTER(_WPack), P]),
         "sharq_prepare": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P]),
         "sharq_linear": (I, [ctypes.POINTER(_Prep), ctypes.POINTER(_WPack), P, I, P]),
-        "sharq_quantize_dense": (I, [P, I, I, P, F, I, P, P, P, P]),
-        "sharq_linear_dense": (I, [P, P, P, I, I, ctypes.POINTER(_WPack), P, I, P]),
+        "sharq_quantize_dense": (I, [P, I, I, P, F, I, P, P, P]),
+        "sharq_linear_dense": (I, [P, P, I, I, ctypes.POINTER(_WPack), P, I, P]),
         "sharq_device_status": (I, [P]),
         "sharq_set_wait_limit": (None, [ctypes.c_longlong]),
         "sharq_last_error": (ctypes.c_char_p, []),
@@ -75,7 +77,23 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     return lib
 
 
-lib = _load()
+class _Lib:
+    """The loaded libsharq.so, opened on first attribute access."""
+    _cdll: ctypes.CDLL | None = None
+
+    def __getattr__(self, name):
+        if _Lib._cdll is None:
+            _Lib._cdll = _load()
+        return getattr(_Lib._cdll, name)
+
+
+lib = _Lib()
+
+
+def load() -> ctypes.CDLL:
+    """Open libsharq.so now (raises ImportError if it is missing or stale)."""
+    lib.sharq_version  # noqa: B018  (attribute access loads the library)
+    return _Lib._cdll
 
 
 def last_error() -> str:
@@ -104,12 +122,8 @@ def _fmt(fmt) -> int:
 # ------------------------------------------------------------------ buffer holders
 @dataclass
 class Prep:
-    """A prepared activation: the six device buffers of ``sharq_prep`` and the C struct."""
-    sparse_codes: torch.Tensor
-    sparse_meta: torch.Tensor
-    sparse_scales: torch.Tensor
-    resid_codes: torch.Tensor
-    resid_scales: torch.Tensor
+    """A prepared activation: the tiled operand, the row scales and the C struct."""
+    tiles: torch.Tensor
     row_scale: torch.Tensor
     tokens: int
     k: int
@@ -121,18 +135,15 @@ class Prep:
 
     def struct(self) -> _Prep:
         if self.c is None:
-            self.c = _Prep(self.sparse_codes.data_ptr(), self.sparse_meta.data_ptr(), self.sparse_scales.data_ptr(),
-                           self.resid_codes.data_ptr(), self.resid_scales.data_ptr(), self.row_scale.data_ptr(),
-                           self.tokens, self.k, self.nm_n, self.nm_m, self.unit, self.fmt)
+            self.c = _Prep(self.tiles.data_ptr(), self.row_scale.data_ptr(), self.tokens, self.k, self.nm_n,
+                           self.nm_m, self.unit, self.fmt)
         return self.c
 
 
 @dataclass
 class WPack:
-    """A packed weight: codes, the two scale views and the tensor scale."""
-    codes: torch.Tensor
-    scales_sparse: torch.Tensor
-    scales_dense: torch.Tensor
+    """A packed weight: the tiled operand (codes and both scale views) and the tensor scale."""
+    tiles: torch.Tensor
     tensor_scale: torch.Tensor
     n_out: int
     k: int
@@ -141,23 +152,27 @@ class WPack:
 
     def struct(self) -> _WPack:
         if self.c is None:
-            self.c = _WPack(self.codes.data_ptr(), self.scales_sparse.data_ptr(), self.scales_dense.data_ptr(),
-                            self.tensor_scale.data_ptr(), self.n_out, self.k, self.fmt)
+            self.c = _WPack(self.tiles.data_ptr(), self.tensor_scale.data_ptr(), self.n_out, self.k, self.fmt)
         return self.c
 
 
-def sharq_prep_buffer_sizes(tokens: int, k: int, nm_n: int, nm_m: int, unit: int, fmt) -> list[int]:
-    sizes = (ctypes.c_size_t * 6)()
-    if lib.sharq_prep_buffer_sizes(tokens, k, nm_n, nm_m, unit, _fmt(fmt), sizes) == 0:
+def _sizes(fn, *args) -> list[int]:
+    sizes = (ctypes.c_size_t * 2)()
+    if fn(*args, sizes) == 0:
         raise SharqError(SHARQ_ERR_INVALID_ARG, last_error())
     return list(sizes)
+
+
+def sharq_prep_buffer_sizes(tokens: int, k: int, nm_n: int, nm_m: int, unit: int, fmt) -> list[int]:
+    return _sizes(lib.sharq_prep_buffer_sizes, tokens, k, nm_n, nm_m, unit, _fmt(fmt))
+
+
+def sharq_dense_buffer_sizes(tokens: int, k: int, fmt) -> list[int]:
+    return _sizes(lib.sharq_dense_buffer_sizes, tokens, k, _fmt(fmt))
 
 
 def sharq_wpack_buffer_sizes(n_out: int, k: int, fmt) -> list[int]:
-    sizes = (ctypes.c_size_t * 4)()
-    if lib.sharq_wpack_buffer_sizes(n_out, k, _fmt(fmt), sizes) == 0:
-        raise SharqError(SHARQ_ERR_INVALID_ARG, last_error())
-    return list(sizes)
+    return _sizes(lib.sharq_wpack_buffer_sizes, n_out, k, _fmt(fmt))
 
 
 def _bytes(n: int, device) -> torch.Tensor:
@@ -168,15 +183,13 @@ def _bytes(n: int, device) -> torch.Tensor:
 def alloc_prep(tokens: int, k: int, nm_n: int = 2, nm_m: int = 4, unit: int = UNIT_PAIR, fmt="nvfp4",
                device="cuda") -> Prep:
     s = sharq_prep_buffer_sizes(tokens, k, nm_n, nm_m, unit, fmt)
-    return Prep(_bytes(s[0], device), _bytes(s[1], device), _bytes(s[2], device), _bytes(s[3], device),
-                _bytes(s[4], device), torch.empty(tokens, dtype=torch.float32, device=device),
+    return Prep(_bytes(s[0], device), torch.empty(tokens, dtype=torch.float32, device=device),
                 tokens, k, nm_n, nm_m, unit, _fmt(fmt))
 
 
 def alloc_wpack(n_out: int, k: int, fmt="nvfp4", device="cuda") -> WPack:
     s = sharq_wpack_buffer_sizes(n_out, k, fmt)
-    return WPack(_bytes(s[0], device), _bytes(s[1], device), _bytes(s[2], device),
-                 torch.empty(4, dtype=torch.float32, device=device), n_out, k, _fmt(fmt))
+    return WPack(_bytes(s[0], device), torch.empty(4, dtype=torch.float32, device=device), n_out, k, _fmt(fmt))
 
 
 # ------------------------------------------------------------------ the calls
@@ -208,7 +221,7 @@ def sharq_linear(prep: Prep, w: WPack, y: torch.Tensor | None = None, out_dtype=
                  stream=None) -> torch.Tensor:
     """Y [tokens, n_out] = sparse FP4 GEMM (backbone) + dense FP4 GEMM (residual), one output."""
     if y is None:
-        y = torch.empty(prep.tokens, w.n_out, dtype=out_dtype, device=prep.resid_codes.device)
+        y = torch.empty(prep.tokens, w.n_out, dtype=out_dtype, device=prep.tiles.device)
     code = SHARQ_OUT_F32 if y.dtype == torch.float32 else SHARQ_OUT_BF16
     _check(lib.sharq_linear(ctypes.byref(prep.struct()), ctypes.byref(w.struct()), _ptr(y), code, _stream(stream)))
     return y
@@ -216,8 +229,8 @@ def sharq_linear(prep: Prep, w: WPack, y: torch.Tensor | None = None, out_dtype=
 
 @dataclass
 class DenseQ:
-    codes: torch.Tensor
-    scales: torch.Tensor
+    """A dense-quantized activation: the tiled operand and the row scales."""
+    tiles: torch.Tensor
     row_scale: torch.Tensor
     tokens: int
     k: int
@@ -230,11 +243,11 @@ def sharq_quantize_dense(x: torch.Tensor, gamma: torch.Tensor | None = None, eps
     assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous()
     tokens, k = x.shape
     if out is None:
-        s = sharq_prep_buffer_sizes(tokens, k, 2, 4, UNIT_PAIR, fmt)
-        out = DenseQ(_bytes(s[3], x.device), _bytes(s[4], x.device),
-                     torch.empty(tokens, dtype=torch.float32, device=x.device), tokens, k, _fmt(fmt))
+        s = sharq_dense_buffer_sizes(tokens, k, fmt)
+        out = DenseQ(_bytes(s[0], x.device), torch.empty(tokens, dtype=torch.float32, device=x.device), tokens, k,
+                     _fmt(fmt))
     _check(lib.sharq_quantize_dense(_ptr(x), tokens, k, _ptr(gamma), ctypes.c_float(eps), _fmt(fmt),
-                                    _ptr(out.codes), _ptr(out.scales), _ptr(out.row_scale), _stream(stream)))
+                                    _ptr(out.tiles), _ptr(out.row_scale), _stream(stream)))
     return out
 
 
@@ -242,10 +255,10 @@ def sharq_linear_dense(q: DenseQ, w: WPack, y: torch.Tensor | None = None, out_d
                        stream=None) -> torch.Tensor:
     """The dense FP4 baseline GEMM against the weight's dense-path scale view."""
     if y is None:
-        y = torch.empty(q.tokens, w.n_out, dtype=out_dtype, device=q.codes.device)
+        y = torch.empty(q.tokens, w.n_out, dtype=out_dtype, device=q.tiles.device)
     code = SHARQ_OUT_F32 if y.dtype == torch.float32 else SHARQ_OUT_BF16
-    _check(lib.sharq_linear_dense(_ptr(q.codes), _ptr(q.scales), _ptr(q.row_scale), q.tokens, q.k,
-                                  ctypes.byref(w.struct()), _ptr(y), code, _stream(stream)))
+    _check(lib.sharq_linear_dense(_ptr(q.tiles), _ptr(q.row_scale), q.tokens, q.k, ctypes.byref(w.struct()),
+                                  _ptr(y), code, _stream(stream)))
     return y
 
 

@@ -28,8 +28,6 @@ int cuda_fail(cudaError_t e, const char *what) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-int block_of(int fmt) { return fmt == SHARQ_NVFP4 ? 16 : 32; }
-
 bool valid_fmt(int fmt) { return fmt == SHARQ_NVFP4 || fmt == SHARQ_MXFP4; }
 
 // Pattern checks shared by sizes and prepare. Returns 0 or a status.
@@ -55,49 +53,46 @@ extern "C" {
 
 const char *sharq_last_error(void) { return g_err; }
 
-int sharq_version(void) { return 100; }
+int sharq_version(void) { return 200; }
 
 void sharq_set_wait_limit(long long spins) { g_wait_limit = spins; }
 
-size_t sharq_prep_buffer_sizes(int tokens, int k, int nm_n, int nm_m, int unit, int fmt, size_t sizes[6]) {
+size_t sharq_prep_buffer_sizes(int tokens, int k, int nm_n, int nm_m, int unit, int fmt, size_t sizes[2]) {
   if (!sizes) { fail(SHARQ_ERR_INVALID_ARG, "sizes is null"); return 0; }
   if (!valid_fmt(fmt)) { fail(SHARQ_ERR_INVALID_ARG, "unknown fmt %d", fmt); return 0; }
   if (check_shape(tokens, k, "tokens") || check_pattern(nm_n, nm_m, unit)) return 0;
-  const size_t T = tokens, K = k, Tp = sharq::round_up(tokens, 256), B = block_of(fmt);
-  const size_t stored = K * nm_n / nm_m;
-  const size_t slab_span = 32u * nm_m * unit;
-  sizes[0] = T * stored / 2;            // sparse codes
-  sizes[1] = (K / slab_span) * Tp * 16;  // metadata
-  sizes[2] = Tp * (stored / B);          // sparse scales
-  sizes[3] = T * K / 2;                  // residual codes
-  sizes[4] = Tp * (K / B);               // residual scales
-  sizes[5] = T * 4;                      // row scales
-  size_t s = 0;
-  for (int i = 0; i < 6; ++i) s += sizes[i];
-  return s;
+  const sharq::ActTile A = sharq::act_tile(fmt, unit, true);
+  sizes[0] = (size_t)(sharq::round_up(tokens, 256) / 128) * (k / 256) * A.bytes;  // tiles
+  sizes[1] = (size_t)tokens * 4;                                                    // row scales
+  return sizes[0] + sizes[1];
 }
 
-size_t sharq_wpack_buffer_sizes(int n_out, int k, int fmt, size_t sizes[4]) {
+size_t sharq_dense_buffer_sizes(int tokens, int k, int fmt, size_t sizes[2]) {
+  if (!sizes) { fail(SHARQ_ERR_INVALID_ARG, "sizes is null"); return 0; }
+  if (!valid_fmt(fmt)) { fail(SHARQ_ERR_INVALID_ARG, "unknown fmt %d", fmt); return 0; }
+  if (check_shape(tokens, k, "tokens")) return 0;
+  const sharq::ActTile A = sharq::act_tile(fmt, 2, false);
+  sizes[0] = (size_t)(sharq::round_up(tokens, 256) / 128) * (k / 256) * A.bytes;
+  sizes[1] = (size_t)tokens * 4;
+  return sizes[0] + sizes[1];
+}
+
+size_t sharq_wpack_buffer_sizes(int n_out, int k, int fmt, size_t sizes[2]) {
   if (!sizes) { fail(SHARQ_ERR_INVALID_ARG, "sizes is null"); return 0; }
   if (!valid_fmt(fmt)) { fail(SHARQ_ERR_INVALID_ARG, "unknown fmt %d", fmt); return 0; }
   if (check_shape(n_out, k, "n_out")) return 0;
   if (n_out % 16) { fail(SHARQ_ERR_INVALID_ARG, "n_out must be a multiple of 16 (got %d)", n_out); return 0; }
-  const size_t N = n_out, K = k, Np = sharq::round_up(n_out, 128), B = block_of(fmt);
-  sizes[0] = N * K / 2;
-  sizes[1] = Np * (K / (2 * B));
-  sizes[2] = Np * (K / B);
-  sizes[3] = 2 * sizeof(float);
-  return sizes[0] + sizes[1] + sizes[2] + sizes[3];
+  sizes[0] = (size_t)(sharq::round_up(n_out, 256) / 128) * (k / 256) * sharq::w_tile(fmt).bytes;
+  sizes[1] = 2 * sizeof(float);
+  return sizes[0] + sizes[1];
 }
 
 int sharq_pack_weight(const void *w, int n_out, int k, int fmt, sharq_wpack *out, void *stream) {
   if (!w || !out) return fail(SHARQ_ERR_INVALID_ARG, "null weight or output struct");
-  size_t sz[4];
+  size_t sz[2];
   if (!sharq_wpack_buffer_sizes(n_out, k, fmt, sz)) return SHARQ_ERR_INVALID_ARG;
-  if (!out->codes || !out->scales_sparse || !out->scales_dense || !out->tensor_scale)
-    return fail(SHARQ_ERR_INVALID_ARG, "null output buffer in sharq_wpack");
-  if (!aligned16(w) || !aligned16(out->codes) || !aligned16(out->scales_sparse) || !aligned16(out->scales_dense) ||
-      !aligned16(out->tensor_scale))
+  if (!out->tiles || !out->tensor_scale) return fail(SHARQ_ERR_INVALID_ARG, "null output buffer in sharq_wpack");
+  if (!aligned16(w) || !aligned16(out->tiles) || !aligned16(out->tensor_scale))
     return fail(SHARQ_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
   out->n_out = n_out;
   out->k = k;
@@ -106,10 +101,8 @@ int sharq_pack_weight(const void *w, int n_out, int k, int fmt, sharq_wpack *out
   p.w = static_cast<const uint16_t *>(w);
   p.N = n_out;
   p.K = k;
-  p.N_pad = sharq::round_up(n_out, 128);
-  p.codes = static_cast<uint8_t *>(out->codes);
-  p.sc_sparse = static_cast<uint8_t *>(out->scales_sparse);
-  p.sc_dense = static_cast<uint8_t *>(out->scales_dense);
+  p.N_pad = sharq::round_up(n_out, 256);
+  p.tiles = static_cast<uint8_t *>(out->tiles);
   p.tensor_scale = out->tensor_scale;
   cudaError_t e = sharq::launch_pack(p, fmt, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "sharq_pack_weight");
@@ -118,19 +111,15 @@ int sharq_pack_weight(const void *w, int n_out, int k, int fmt, sharq_wpack *out
 }
 
 static int prepare_common(const void *x, int tokens, int k, const void *gamma, float eps, int fmt, bool dense,
-                          int nm_n, int nm_m, int unit, uint8_t *sp_codes, uint8_t *meta, uint8_t *sp_scales,
-                          uint8_t *res_codes, uint8_t *res_scales, float *row_scale, cudaStream_t st) {
+                          int unit, uint8_t *tiles, float *row_scale, cudaStream_t st) {
   if (!x) return fail(SHARQ_ERR_INVALID_ARG, "x is null");
   if (!valid_fmt(fmt)) return fail(SHARQ_ERR_INVALID_ARG, "unknown fmt %d", fmt);
   if (int s = check_shape(tokens, k, "tokens")) return s;
   if (k > 32768) return fail(SHARQ_ERR_INVALID_ARG, "k must be <= 32768 for the preparation kernel (got %d)", k);
   if (((uintptr_t)x & 31u) || ((uintptr_t)gamma & 31u))
     return fail(SHARQ_ERR_INVALID_ARG, "x and gamma must be 32-byte aligned (256-bit loads)");
-  if (!res_codes || !res_scales || !row_scale) return fail(SHARQ_ERR_INVALID_ARG, "null output buffer");
-  if (!dense && (!sp_codes || !meta || !sp_scales)) return fail(SHARQ_ERR_INVALID_ARG, "null output buffer");
-  const void *bufs[6] = {sp_codes, meta, sp_scales, res_codes, res_scales, row_scale};
-  for (int i = dense ? 3 : 0; i < 6; ++i)
-    if (!aligned16(bufs[i])) return fail(SHARQ_ERR_INVALID_ARG, "output buffer %d is not 16-byte aligned", i);
+  if (!tiles || !row_scale) return fail(SHARQ_ERR_INVALID_ARG, "null output buffer");
+  if (!aligned16(tiles) || !aligned16(row_scale)) return fail(SHARQ_ERR_INVALID_ARG, "output buffers must be 16-byte aligned");
   if (gamma && !(eps >= 0.f)) return fail(SHARQ_ERR_INVALID_ARG, "eps must be >= 0");
   sharq::PrepParams p;
   p.x = static_cast<const uint16_t *>(x);
@@ -139,15 +128,8 @@ static int prepare_common(const void *x, int tokens, int k, const void *gamma, f
   p.T = tokens;
   p.K = k;
   p.T_pad = sharq::round_up(tokens, 256);
-  p.sp_codes = sp_codes;
-  p.meta = meta;
-  p.sp_scales = sp_scales;
-  p.res_codes = res_codes;
-  p.res_scales = res_scales;
+  p.tiles = tiles;
   p.row_scale = row_scale;
-  const int B = block_of(fmt);
-  p.n_sf_res = k / B;
-  p.n_sf_sp = dense ? 0 : k * nm_n / nm_m / B;
   cudaError_t e = sharq::launch_prep(p, fmt, unit, gamma != nullptr, dense, st);
   if (e != cudaSuccess) return cuda_fail(e, dense ? "sharq_quantize_dense" : "sharq_prepare");
   g_err[0] = 0;
@@ -158,10 +140,8 @@ int sharq_prepare(const void *x, int tokens, int k, const void *gamma, float eps
                   int fmt, sharq_prep *out, void *stream) {
   if (!out) return fail(SHARQ_ERR_INVALID_ARG, "output struct is null");
   if (int s = check_pattern(nm_n, nm_m, unit)) return s;
-  int s = prepare_common(x, tokens, k, gamma, eps, fmt, false, nm_n, nm_m, unit,
-                         static_cast<uint8_t *>(out->sparse_codes), static_cast<uint8_t *>(out->sparse_meta),
-                         static_cast<uint8_t *>(out->sparse_scales), static_cast<uint8_t *>(out->resid_codes),
-                         static_cast<uint8_t *>(out->resid_scales), out->row_scale, static_cast<cudaStream_t>(stream));
+  int s = prepare_common(x, tokens, k, gamma, eps, fmt, false, unit, static_cast<uint8_t *>(out->tiles),
+                         out->row_scale, static_cast<cudaStream_t>(stream));
   if (s == SHARQ_OK) {
     out->tokens = tokens;
     out->k = k;
@@ -173,10 +153,9 @@ int sharq_prepare(const void *x, int tokens, int k, const void *gamma, float eps
   return s;
 }
 
-int sharq_quantize_dense(const void *x, int tokens, int k, const void *gamma, float eps, int fmt, void *codes,
-                         void *scales, float *row_scale, void *stream) {
-  return prepare_common(x, tokens, k, gamma, eps, fmt, true, 4, 4, 1, nullptr, nullptr, nullptr,
-                        static_cast<uint8_t *>(codes), static_cast<uint8_t *>(scales), row_scale,
+int sharq_quantize_dense(const void *x, int tokens, int k, const void *gamma, float eps, int fmt, void *tiles,
+                         float *row_scale, void *stream) {
+  return prepare_common(x, tokens, k, gamma, eps, fmt, true, 2, static_cast<uint8_t *>(tiles), row_scale,
                         static_cast<cudaStream_t>(stream));
 }
 
@@ -185,10 +164,8 @@ static int check_wpack(const sharq_wpack *w) {
   if (!valid_fmt(w->fmt)) return fail(SHARQ_ERR_INVALID_ARG, "weight pack has unknown fmt %d", w->fmt);
   if (int s = check_shape(w->n_out, w->k, "n_out")) return s;
   if (w->n_out % 16) return fail(SHARQ_ERR_INVALID_ARG, "n_out must be a multiple of 16");
-  if (!w->codes || !w->scales_sparse || !w->scales_dense || !w->tensor_scale)
-    return fail(SHARQ_ERR_INVALID_ARG, "null buffer in weight pack");
-  if (!aligned16(w->codes) || !aligned16(w->scales_sparse) || !aligned16(w->scales_dense))
-    return fail(SHARQ_ERR_INVALID_ARG, "weight buffers must be 16-byte aligned");
+  if (!w->tiles || !w->tensor_scale) return fail(SHARQ_ERR_INVALID_ARG, "null buffer in weight pack");
+  if (!aligned16(w->tiles)) return fail(SHARQ_ERR_INVALID_ARG, "weight buffers must be 16-byte aligned");
   return 0;
 }
 
@@ -214,60 +191,48 @@ int sharq_linear(const sharq_prep *a, const sharq_wpack *w, void *y, int out_dty
     return fail(SHARQ_ERR_UNSUPPORTED,
                 "the sparse FP4 MMA executes pattern 2:4 over pairs (unit 2); got %d:%d unit %d", a->nm_n, a->nm_m,
                 a->unit);
-  if (!a->sparse_codes || !a->sparse_meta || !a->sparse_scales || !a->resid_codes || !a->resid_scales ||
-      !a->row_scale)
-    return fail(SHARQ_ERR_INVALID_ARG, "null buffer in prep");
-  const void *bufs[7] = {a->sparse_codes, a->sparse_meta, a->sparse_scales, a->resid_codes, a->resid_scales,
-                         a->row_scale, y};
-  for (int i = 0; i < 7; ++i)
-    if (!aligned16(bufs[i])) return fail(SHARQ_ERR_INVALID_ARG, "buffer %d is not 16-byte aligned", i);
+  if (!a->tiles || !a->row_scale) return fail(SHARQ_ERR_INVALID_ARG, "null buffer in prep");
+  if (!aligned16(a->tiles) || !aligned16(a->row_scale) || !aligned16(y))
+    return fail(SHARQ_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
   sharq::GemmParams g;
-  g.a_res = static_cast<const uint8_t *>(a->resid_codes);
-  g.a_sp = static_cast<const uint8_t *>(a->sparse_codes);
-  g.meta = static_cast<const uint8_t *>(a->sparse_meta);
-  g.sfa_res = static_cast<const uint8_t *>(a->resid_scales);
-  g.sfa_sp = static_cast<const uint8_t *>(a->sparse_scales);
+  memset(&g, 0, sizeof g);
+  g.a_tiles = static_cast<const uint8_t *>(a->tiles);
   g.row_scale = a->row_scale;
-  g.b = static_cast<const uint8_t *>(w->codes);
-  g.sfb_dense = static_cast<const uint8_t *>(w->scales_dense);
-  g.sfb_sparse = static_cast<const uint8_t *>(w->scales_sparse);
+  g.w_tiles = static_cast<const uint8_t *>(w->tiles);
   g.tensor_scale = w->tensor_scale;
   g.y = y;
   g.T = a->tokens;
   g.N = w->n_out;
   g.K = a->k;
   g.T_pad = sharq::round_up(a->tokens, 256);
-  g.N_pad = sharq::round_up(w->n_out, 128);
+  g.N_pad = sharq::round_up(w->n_out, 256);
   g.fmt = a->fmt;
   g.out_f32 = out_dtype == SHARQ_OUT_F32;
   g.sparse = 1;
   return run_gemm(g, "sharq_linear", static_cast<cudaStream_t>(stream));
 }
 
-int sharq_linear_dense(const void *codes, const void *scales, const float *row_scale, int tokens, int k,
-                       const sharq_wpack *w, void *y, int out_dtype, void *stream) {
-  if (!codes || !scales || !row_scale || !y) return fail(SHARQ_ERR_INVALID_ARG, "null buffer");
+int sharq_linear_dense(const void *tiles, const float *row_scale, int tokens, int k, const sharq_wpack *w, void *y,
+                       int out_dtype, void *stream) {
+  if (!tiles || !row_scale || !y) return fail(SHARQ_ERR_INVALID_ARG, "null buffer");
   if (int s = check_wpack(w)) return s;
   if (int s = check_shape(tokens, k, "tokens")) return s;
   if (k != w->k) return fail(SHARQ_ERR_INVALID_ARG, "k mismatch: activation %d, weight %d", k, w->k);
   if (out_dtype != SHARQ_OUT_BF16 && out_dtype != SHARQ_OUT_F32) return fail(SHARQ_ERR_INVALID_ARG, "bad out_dtype");
-  if (!aligned16(codes) || !aligned16(scales) || !aligned16(row_scale) || !aligned16(y))
+  if (!aligned16(tiles) || !aligned16(row_scale) || !aligned16(y))
     return fail(SHARQ_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
   sharq::GemmParams g;
   memset(&g, 0, sizeof g);
-  g.a_res = static_cast<const uint8_t *>(codes);
-  g.sfa_res = static_cast<const uint8_t *>(scales);
+  g.a_tiles = static_cast<const uint8_t *>(tiles);
   g.row_scale = row_scale;
-  g.b = static_cast<const uint8_t *>(w->codes);
-  g.sfb_dense = static_cast<const uint8_t *>(w->scales_dense);
-  g.sfb_sparse = static_cast<const uint8_t *>(w->scales_sparse);
+  g.w_tiles = static_cast<const uint8_t *>(w->tiles);
   g.tensor_scale = w->tensor_scale;
   g.y = y;
   g.T = tokens;
   g.N = w->n_out;
   g.K = k;
   g.T_pad = sharq::round_up(tokens, 256);
-  g.N_pad = sharq::round_up(w->n_out, 128);
+  g.N_pad = sharq::round_up(w->n_out, 256);
   g.fmt = w->fmt;
   g.out_f32 = out_dtype == SHARQ_OUT_F32;
   g.sparse = 0;

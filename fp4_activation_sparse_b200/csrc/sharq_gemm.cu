@@ -10,17 +10,20 @@
 // sm_100a design. A cluster of two CTAs on the two SMs of a TPC works on one 256 x 256
 // output tile with cta_group::2 MMAs (M = 256, N = 256): each CTA loads its own 128
 // activation rows and half of the weight tile (128 rows), so every weight byte crosses
-// into shared memory once per pair. Persistent over tiles, K-tiles of 256, four stages.
-//   warp 0      TMA producer (both CTAs): residual codes (SW128), compressed backbone codes
-//               (SW64), weight codes (SW128), backbone metadata and the four scale tiles
-//               (pre-tiled 128x4 atoms); every load completes on the leader CTA's barrier.
-//               Each weight tile feeds both MMAs.
+// into shared memory once per pair. Persistent over tiles, K steps of 256, four stages.
+// Both operands are pre-tiled in global memory (chunks of 128 rows x 256 K that are the
+// exact shared-memory image: swizzled codes, metadata, 128x4 scale atoms), so a stage is
+// two bulk tensor copies per CTA -- the copy count per stage, not the bytes, is what
+// bounds a TMA-fed pipeline at this tile size.
+//   warp 0      TMA producer (both CTAs): the activation chunk and the weight chunk of the
+//               K step; every load completes on the leader CTA's barrier.
 //   warp 1      TMEM owner (both CTAs) and, in the leader, the single MMA-issuing thread:
 //               tcgen05.cp moves scales and metadata to tensor memory, then two
 //               tcgen05.mma.sp (K=128 logical, pairwise 4:8) and four dense tcgen05.mma
 //               (K=64) accumulate into one fp32 accumulator of 128 x 256 per CTA. Both
 //               paths carry the same per-row scale s_x, so one accumulator holds their sum.
-//               Commits arrive on both CTAs' barriers (multicast commit).
+//               Each weight chunk feeds both MMAs. Commits arrive on both CTAs' barriers
+//               (multicast commit).
 //   warps 2..9  epilogue (both CTAs): tcgen05.ld, y = acc * s_x[row] * s_w, bf16/fp32 stores.
 // Every mbarrier wait is bounded by a time limit; on expiry the CTA records a status word,
 // stops issuing, drains (bounded) what it issued, frees TMEM and exits.
@@ -40,7 +43,6 @@ namespace {
 
 constexpr int BM = 128;   // activation rows per CTA (256 per pair)
 constexpr int BN = 256;   // output columns per pair tile
-constexpr int BNH = 128;  // weight rows loaded per CTA
 constexpr int BK = 256;   // logical K per stage
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;
@@ -52,20 +54,21 @@ constexpr uint32_t kScaleBufCols = 80;  // per K-tile parity: meta 4, SFA_sp 8, 
 // test lowers the limit of the ordinary waits.
 constexpr uint64_t kDrainLimitNs = 4000000000ull;
 
-// shared-memory stage layout (bytes), identical in both CTAs
-constexpr int OFF_ARES = 0;         // 128 rows x 128 B, SW128
-constexpr int OFF_B = 16384;        // 128 weight rows x 128 B, SW128
-constexpr int OFF_ASP = 32768;      // 128 rows x 64 B, SW64
-constexpr int OFF_META = 40960;     // 128 rows x 16 B
-constexpr int OFF_SFA_RES = 43008;  // up to 4 atoms
-constexpr int OFF_SFA_SP = 45056;   // up to 2 atoms
-constexpr int OFF_SFB_RES = 46080;  // n-block 0 at +0, n-block 1 at +2048
-constexpr int OFF_SFB_SP = 50176;   // n-block 0 at +0, n-block 1 at +1024
-constexpr int kStageBytes = 52224;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align slack*/ + 256 /*barriers*/;
+// shared-memory stage: the activation chunk, then the weight chunk (identical in both CTAs)
+template <bool MX, bool SPARSE>
+struct Stage {
+  static constexpr ActTile A = act_tile(MX ? 1 : 0, 2, SPARSE);
+  static constexpr WTile W = w_tile(MX ? 1 : 0);
+  static constexpr int kW = A.bytes;  // 1024-aligned: the weight codes are 128-byte swizzled
+  static constexpr int kBytes = A.bytes + W.bytes;
+};
+constexpr int kMaxStageBytes = 52224;  // NVFP4 SharQ: 29696 + 22528
+constexpr int kSmemBytes = kStages * kMaxStageBytes + 1024 /*align slack*/ + 256 /*barriers*/;
+static_assert(Stage<false, true>::kBytes <= kMaxStageBytes && Stage<true, true>::kBytes <= kMaxStageBytes, "stage");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 struct __align__(64) TmaMaps {
-  CUtensorMap a_res, a_sp, b, meta, sfa_res, sfa_sp, sfb_res, sfb_sp;
+  CUtensorMap act, w;  // both: rows of 1024 bytes (256 x u32), one box = one chunk
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -251,15 +254,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// atoms of one K-tile for a scale tensor whose scale covers `span` K positions
-__host__ __device__ constexpr int atoms_per_ktile(int span) { return BK / span / 4; }
-
 template <bool MX, bool SPARSE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     sharq_gemm_kernel(const __grid_constant__ TmaMaps maps, GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kMaxStageBytes);
   // bars: full[kStages], empty[kStages], acc_full, acc_empty, drain
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kStages + 3);
   volatile uint32_t *abort_flag = tmem_slot + 1;
@@ -273,9 +273,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
   const uint32_t acc_full = bar0 + 8u * (2 * kStages), acc_empty = acc_full + 8, drain_bar = acc_full + 16;
 
-  const int B = MX ? 32 : 16;               // dense block
-  const int span_res = B, span_sp = 2 * B;  // K positions per scale
-  const int apt_res = atoms_per_ktile(span_res), apt_sp = atoms_per_ktile(span_sp);
+  using L = Stage<MX, SPARSE>;
+  constexpr int apt_res = atoms_res(MX ? 1 : 0), apt_sp = atoms_sp(MX ? 1 : 0);
+  constexpr int kStageBytes = L::kBytes;
   const int num_m = (p.T + 2 * BM - 1) / (2 * BM), num_n = (p.N + BN - 1) / BN, num_k = p.K / BK;
   const int num_tiles = num_m * num_n;
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
@@ -293,16 +293,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0 && lane == 0) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.a_res) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.b) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.sfa_res) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.sfb_res) : "memory");
-    if (SPARSE) {
-      asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.a_sp) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.meta) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.sfa_sp) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.sfb_sp) : "memory");
-    }
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.act) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.w) : "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -325,33 +317,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
         const int m0 = (tile % num_m) * (2 * BM) + (int)rank * BM;  // this CTA's activation rows
         const int n0 = (tile / num_m) * BN;                          // the pair's output columns
-        const int nb_valid = min(2, (p.N_pad - n0) / 128);            // scale n-blocks inside the padded weight
-        const int mb = m0 / 128;
+        const int a_row0 = (m0 / 128) * num_k * (L::A.bytes / 1024);  // chunk rows of 1024 bytes
+        const int w_row0 = (n0 / 128 + (int)rank) * num_k * (L::W.bytes / 1024);
         for (int kt = 0; kt < num_k; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, limit, abort_flag)) { ok = false; break; }
           const uint32_t st = smem0 + stage * kStageBytes;
           if (leader) {
-            uint32_t bytes = 16384 + 16384 + apt_res * 512 + nb_valid * apt_res * 512;
-            if (SPARSE) bytes += 8192 + 2048 + apt_sp * 512 + nb_valid * apt_sp * 512;
-            mbar_expect_tx(full_bar(stage), 2 * bytes);
+            mbar_expect_tx(full_bar(stage), 2u * kStageBytes);
             armed |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           }
           const uint32_t fb = full_leader0 + 8u * stage;
-          tma_load_2d(st + OFF_ARES, &maps.a_res, kt * 128, m0, fb);
-          tma_load_2d(st + OFF_B, &maps.b, kt * 128, n0 + (int)rank * BNH, fb);
-          tma_load_2d(st + OFF_SFA_RES, &maps.sfa_res, 0, mb * (p.K / span_res / 4) + kt * apt_res, fb);
-          for (int i = 0; i < nb_valid; ++i)
-            tma_load_2d(st + OFF_SFB_RES + i * 2048, &maps.sfb_res, 0,
-                        (n0 / 128 + i) * (p.K / span_res / 4) + kt * apt_res, fb);
-          if (SPARSE) {
-            tma_load_2d(st + OFF_ASP, &maps.a_sp, kt * 64, m0, fb);
-            tma_load_2d(st + OFF_META, &maps.meta, 0, kt * p.T_pad + m0, fb);
-            tma_load_2d(st + OFF_SFA_SP, &maps.sfa_sp, 0, mb * (p.K / span_sp / 4) + kt * apt_sp, fb);
-            for (int i = 0; i < nb_valid; ++i)
-              tma_load_2d(st + OFF_SFB_SP + i * 1024, &maps.sfb_sp, 0,
-                          (n0 / 128 + i) * (p.K / span_sp / 4) + kt * apt_sp, fb);
-          }
+          tma_load_2d(st, &maps.act, 0, a_row0 + kt * (L::A.bytes / 1024), fb);
+          tma_load_2d(st + L::kW, &maps.w, 0, w_row0 + kt * (L::W.bytes / 1024), fb);
           issued = true;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
@@ -388,20 +366,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t sbuf = tmem + kAccCols + (kt & 1) * kScaleBufCols;
           const uint32_t t_meta = sbuf, t_sfa_sp = sbuf + 4, t_sfa_res = sbuf + 12, t_sfb_sp = sbuf + 28,
                          t_sfb_res = sbuf + 44;
-          // scales and metadata: shared memory -> tensor memory (both CTAs)
+          constexpr int kA = 0, kW = L::kW;
+          // scales and metadata: shared memory -> tensor memory (both CTAs). The weight
+          // chunk holds the scales of both 128-row halves of the pair's 256 columns.
 #pragma unroll
           for (int a = 0; a < apt_res; ++a) {
-            tc_cp_atom(t_sfa_res + 4 * a, dsc(kDescNone, st4 + (OFF_SFA_RES + a * 512) / 16));
-            tc_cp_atom(t_sfb_res + 8 * a, dsc(kDescNone, st4 + (OFF_SFB_RES + a * 512) / 16));
-            tc_cp_atom(t_sfb_res + 8 * a + 4, dsc(kDescNone, st4 + (OFF_SFB_RES + 2048 + a * 512) / 16));
+            tc_cp_atom(t_sfa_res + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_res + a * 512) / 16));
+            tc_cp_atom(t_sfb_res + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_res + a * 512) / 16));
+            tc_cp_atom(t_sfb_res + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_res + (apt_res + a) * 512) / 16));
           }
           if (SPARSE) {
-            tc_cp_128x128(t_meta, dsc(kDescNone, st4 + OFF_META / 16));
+            tc_cp_128x128(t_meta, dsc(kDescNone, st4 + (kA + L::A.meta) / 16));
 #pragma unroll
             for (int a = 0; a < apt_sp; ++a) {
-              tc_cp_atom(t_sfa_sp + 4 * a, dsc(kDescNone, st4 + (OFF_SFA_SP + a * 512) / 16));
-              tc_cp_atom(t_sfb_sp + 8 * a, dsc(kDescNone, st4 + (OFF_SFB_SP + a * 512) / 16));
-              tc_cp_atom(t_sfb_sp + 8 * a + 4, dsc(kDescNone, st4 + (OFF_SFB_SP + 1024 + a * 512) / 16));
+              tc_cp_atom(t_sfa_sp + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_sp + a * 512) / 16));
+              tc_cp_atom(t_sfb_sp + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_sp + a * 512) / 16));
+              tc_cp_atom(t_sfb_sp + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_sp + (apt_sp + a) * 512) / 16));
             }
           }
           uint32_t accumulate = kt > 0 ? 1u : 0u;
@@ -412,9 +392,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               // NVFP4: 4 scales per row per MMA (one atom, id 0); MXFP4: 2 (half an atom)
               const uint32_t atom = MX ? (uint32_t)(j >> 1) : (uint32_t)j;
               const uint32_t id = MX ? (uint32_t)(2 * (j & 1)) : 0u;
-              mma_sparse<MX>(acc, dsc(kDescSw64, st4 + (OFF_ASP + 32 * j) / 16),
-                             dsc(kDescSw128, st4 + (OFF_B + 64 * j) / 16), t_meta + 2 * j, idesc_bs(true, MX, id, id),
-                             (t_sfa_sp + 4 * atom) | (id << 30), (t_sfb_sp + 8 * atom) | (id << 30), accumulate);
+              mma_sparse<MX>(acc, dsc(kDescSw64, st4 + (kA + L::A.sp + 32 * j) / 16),
+                             dsc(kDescSw128, st4 + (kW + L::W.b + 64 * j) / 16), t_meta + 2 * j,
+                             idesc_bs(true, MX, id, id), (t_sfa_sp + 4 * atom) | (id << 30),
+                             (t_sfb_sp + 8 * atom) | (id << 30), accumulate);
               accumulate = 1u;
             }
           }
@@ -422,8 +403,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 4; ++j) {  // four dense MMAs of K = 64 (32 bytes of A and B)
             const uint32_t atom = MX ? (uint32_t)(j >> 1) : (uint32_t)j;
             const uint32_t id = MX ? (uint32_t)(2 * (j & 1)) : 0u;
-            mma_dense<MX>(acc, dsc(kDescSw128, st4 + (OFF_ARES + 32 * j) / 16),
-                          dsc(kDescSw128, st4 + (OFF_B + 32 * j) / 16), idesc_bs(false, MX, id, id),
+            mma_dense<MX>(acc, dsc(kDescSw128, st4 + (kA + L::A.res + 32 * j) / 16),
+                          dsc(kDescSw128, st4 + (kW + L::W.b + 32 * j) / 16), idesc_bs(false, MX, id, id),
                           (t_sfa_res + 4 * atom) | (id << 30), (t_sfb_res + 8 * atom) | (id << 30), accumulate);
             accumulate = 1u;
           }
@@ -558,21 +539,15 @@ cudaError_t launch_t(const TmaMaps &maps, const GemmParams &p, cudaStream_t st) 
 cudaError_t launch_gemm(const GemmParams &p, cudaStream_t st, const char **why) {
   TmaMaps maps;
   memset(&maps, 0, sizeof maps);
-  const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8, U32 = CU_TENSOR_MAP_DATA_TYPE_UINT32;
-  const auto NONE = CU_TENSOR_MAP_SWIZZLE_NONE;
-  const int B = p.fmt == kFmtMX ? 32 : 16;
-  const uint64_t atoms_res_a = (uint64_t)(p.T_pad / 128) * (p.K / B / 4);
-  const uint64_t atoms_res_b = (uint64_t)(p.N_pad / 128) * (p.K / B / 4);
-  const uint32_t apt_res = atoms_per_ktile(B), apt_sp = atoms_per_ktile(2 * B);
-  bool ok = make_map(&maps.a_res, p.a_res, U8, (uint64_t)p.K / 2, (uint64_t)p.T, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            make_map(&maps.b, p.b, U8, (uint64_t)p.K / 2, (uint64_t)p.N, 128, BNH, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            make_map(&maps.sfa_res, p.sfa_res, U32, 128, atoms_res_a, 128, apt_res, NONE) &&
-            make_map(&maps.sfb_res, p.sfb_dense, U32, 128, atoms_res_b, 128, apt_res, NONE);
-  if (ok && p.sparse)
-    ok = make_map(&maps.a_sp, p.a_sp, U8, (uint64_t)p.K / 4, (uint64_t)p.T, 64, BM, CU_TENSOR_MAP_SWIZZLE_64B) &&
-         make_map(&maps.meta, p.meta, U32, 4, (uint64_t)(p.K / 256) * p.T_pad, 4, BM, NONE) &&
-         make_map(&maps.sfa_sp, p.sfa_sp, U32, 128, atoms_res_a / 2, 128, apt_sp, NONE) &&
-         make_map(&maps.sfb_sp, p.sfb_sparse, U32, 128, atoms_res_b / 2, 128, apt_sp, NONE);
+  const int fmt = p.fmt == kFmtMX ? 1 : 0;
+  const ActTile A = act_tile(fmt, 2, p.sparse != 0);
+  const WTile W = w_tile(fmt);
+  const uint64_t ks = (uint64_t)p.K / BK;
+  const uint64_t a_rows = (uint64_t)(p.T_pad / 128) * ks * (A.bytes / 1024);
+  const uint64_t w_rows = (uint64_t)(p.N_pad / 128) * ks * (W.bytes / 1024);
+  const auto U32 = CU_TENSOR_MAP_DATA_TYPE_UINT32;
+  const bool ok = make_map(&maps.act, p.a_tiles, U32, 256, a_rows, 256, A.bytes / 1024, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                  make_map(&maps.w, p.w_tiles, U32, 256, w_rows, 256, W.bytes / 1024, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or operand layout rejected)";
     return cudaErrorInvalidValue;

@@ -6,37 +6,66 @@
 
 namespace sharq {
 
+// ---------------------------------------------------------------- tiled operands
+// Activations and weights are stored as chunks of 128 rows x 256 K, one contiguous chunk
+// per (128-row block, 256-K step), chunk-major [row block][K step]. A chunk is the exact
+// shared-memory image the GEMM's tensor-core descriptors and scale copies read, so one
+// bulk copy moves it. Offsets inside a chunk (bytes):
+//   activation, SharQ prep:  res  128 x 128 B residual codes, 128-byte swizzle
+//                            sp   128 x 64 B backbone codes (kept values), 64-byte swizzle
+//                            meta 128 x 16 B metadata (pair unit; element unit: two slabs
+//                                 of 128 x 16 B, 4096 B)
+//                            sf_sp / sf_res  backbone / residual scales as 128x4 atoms
+//   activation, dense quantizer: res codes + sf_res only
+//   weight (128 rows = one half of a 256-row block): b 128 x 128 B codes, 128-byte swizzle;
+//                            sf_sp / sf_res the scales of the whole 256-row block (the
+//                            rows of both halves, block-half-major), so each half's chunk
+//                            carries what a CTA pair's MMA reads for its 256 columns.
+// Chunk sizes are multiples of 1024 bytes.
+struct ActTile {
+  int res, sp, meta, sf_sp, sf_res, bytes;
+};
+struct WTile {
+  int b, sf_sp, sf_res, bytes;
+};
+__host__ __device__ constexpr int tile_round(int a) { return (a + 1023) / 1024 * 1024; }
+// scale atoms (512 B, 4 scales x 128 rows) per 256-K step for 128 rows; fmt 0 = NVFP4, 1 = MXFP4
+__host__ __device__ constexpr int atoms_res(int fmt) { return fmt == 0 ? 4 : 2; }  // one scale per B
+__host__ __device__ constexpr int atoms_sp(int fmt) { return fmt == 0 ? 2 : 1; }   // one scale per 2B
+__host__ __device__ constexpr ActTile act_tile(int fmt, int unit, bool sparse) {
+  return sparse ? ActTile{0, 16384, 24576, 24576 + (unit == 2 ? 2048 : 4096),
+                          24576 + (unit == 2 ? 2048 : 4096) + 512 * atoms_sp(fmt),
+                          tile_round(24576 + (unit == 2 ? 2048 : 4096) + 512 * (atoms_sp(fmt) + atoms_res(fmt)))}
+                : ActTile{0, 0, 0, 0, 16384, tile_round(16384 + 512 * atoms_res(fmt))};
+}
+__host__ __device__ constexpr WTile w_tile(int fmt) {
+  return WTile{0, 16384, 16384 + 1024 * atoms_sp(fmt), 16384 + 1024 * (atoms_sp(fmt) + atoms_res(fmt))};
+}
+// byte offset of (row r in 0..127, scale s of the K step) inside a run of 128x4 atoms
+__host__ __device__ constexpr int atom_pos(int r, int s) { return (s >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (s & 3); }
+
 struct PrepParams {
   const uint16_t *x;      // [T][K] bf16
   const uint16_t *gamma;  // [K] bf16 or null
   float eps;
   int T, K, T_pad;
-  int C;   // 64-element chunks per row
-  int TS;  // threads per row team
-  uint8_t *sp_codes, *meta, *sp_scales, *res_codes, *res_scales;
-  float *row_scale;
-  int n_sf_sp, n_sf_res;  // scales per row of the backbone / residual
+  int KS;  // 256-K steps per row
+  int TS;  // warps per row team
+  uint8_t *tiles;         // activation chunks (act_tile layout)
+  float *row_scale;       // [T]
 };
 
 struct PackParams {
   const uint16_t *w;  // [N][K] bf16
   int N, K, N_pad;
-  uint8_t *codes, *sc_sparse, *sc_dense;
+  uint8_t *tiles;       // weight chunks (w_tile layout)
   float *tensor_scale;  // [0] s_w, [1] amax
 };
 
 struct GemmParams {
-  // activation operands
-  const uint8_t *a_res;       // [T][K/2]
-  const uint8_t *a_sp;        // [T][K/4] (null for the dense-only GEMM)
-  const uint8_t *meta;        // slabs [K/256][T_pad][16]
-  const uint8_t *sfa_res;     // atoms, K/B per row
-  const uint8_t *sfa_sp;      // atoms, K/(2B) per row
+  const uint8_t *a_tiles;     // activation chunks: SharQ prep (sparse) or dense quantizer
   const float *row_scale;     // [T]
-  // weight operands
-  const uint8_t *b;           // [N][K/2]
-  const uint8_t *sfb_dense;   // atoms, K/B per row
-  const uint8_t *sfb_sparse;  // atoms, K/(2B) per row
+  const uint8_t *w_tiles;     // weight chunks
   const float *tensor_scale;  // [0] = s_w
   void *y;                    // [T][N]
   int T, N, K, T_pad, N_pad;

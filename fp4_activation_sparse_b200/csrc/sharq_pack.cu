@@ -10,7 +10,9 @@
 //
 // Launch 1 reduces amax|W| into tensor_scale[1] (float bits of a non-negative value
 // order like unsigned integers, so atomicMax on the bits is a float max). Launch 2
-// quantizes: one thread per (row, 64-element chunk).
+// quantizes: one thread per (row, 64-element piece), writing the tiled weight operand
+// (chunks of 128 rows x 256 K: 128-byte-swizzled codes plus both scale views of the
+// 256-row block, stored in the chunks of both of its halves). Rows N..N_pad-1 are zeroed.
 #include "sharq_common.cuh"
 #include "sharq_internal.h"
 #include "sharq_quant.cuh"
@@ -40,22 +42,44 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *w, size_t n_v
   }
 }
 
+// Scale bytes of one 64-K piece: `sp` (2 NVFP4 / 1 MXFP4 bytes) at sparse-view index s0
+// and `dn` (4 / 2 bytes) at dense-view index d0 of the K step, written for row n into the
+// chunks of both halves of its 256-row block.
+template <int FMT>
+__device__ __forceinline__ void store_scales(const PackParams &p, int n, int ks, int s0, int d0, uint32_t sp,
+                                             uint32_t dn) {
+  constexpr WTile L = w_tile(FMT);
+  const int KS = p.K / 256, r = n & 127, half = (n >> 7) & 1;
+  for (int h = 0; h < 2; ++h) {
+    uint8_t *chunk = p.tiles + ((size_t)(((n >> 8) << 1) + h) * KS + ks) * L.bytes;
+    uint8_t *sp_at = chunk + L.sf_sp + half * 512 * atoms_sp(FMT) + atom_pos(r, s0);
+    uint8_t *dn_at = chunk + L.sf_res + half * 512 * atoms_res(FMT) + atom_pos(r, d0);
+    if (FMT == kFmtNV) {
+      *reinterpret_cast<uint16_t *>(sp_at) = (uint16_t)sp;
+      *reinterpret_cast<uint32_t *>(dn_at) = dn;
+    } else {
+      *sp_at = (uint8_t)sp;
+      *reinterpret_cast<uint16_t *>(dn_at) = (uint16_t)dn;
+    }
+  }
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(128) pack_kernel(PackParams p) {
+  constexpr WTile L = w_tile(FMT);
   const int C = p.K / 64;
   const size_t gid = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
   if (gid >= (size_t)p.N_pad * C) return;
   const int n = (int)(gid / C), c = (int)(gid % C);
-  const int spr_dense = FMT == kFmtNV ? p.K / 16 : p.K / 32;
-  const int spr_sparse = spr_dense / 2;
-  if (n >= p.N) {  // padding rows of the scale atoms
-    if (FMT == kFmtNV) {
-      *reinterpret_cast<uint16_t *>(p.sc_sparse + atom_offset(n, 2 * c, spr_sparse)) = 0;
-      *reinterpret_cast<uint32_t *>(p.sc_dense + atom_offset(n, 4 * c, spr_dense)) = 0u;
-    } else {
-      p.sc_sparse[atom_offset(n, c, spr_sparse)] = 0;
-      *reinterpret_cast<uint16_t *>(p.sc_dense + atom_offset(n, 2 * c, spr_dense)) = 0;
-    }
+  const int ks = c >> 2, c4 = c & 3, r = n & 127;
+  // sparse view: NVFP4 2 scales (of 32 K) per piece, MXFP4 1 (of 64 K); dense view twice as many
+  const int s0 = FMT == kFmtNV ? 2 * c4 : c4, d0 = 2 * s0;
+  uint4 *dst = reinterpret_cast<uint4 *>(p.tiles + ((size_t)(n >> 7) * (p.K / 256) + ks) * L.bytes + L.b + r * 128);
+  const int u0 = 2 * c4;  // 16-byte units u0, u0+1 of the 128-byte row, swizzled with row bits 0..2
+  if (n >= p.N) {  // padding rows
+    store_scales<FMT>(p, n, ks, s0, d0, 0u, 0u);
+    dst[u0 ^ (r & 7)] = make_uint4(0u, 0u, 0u, 0u);
+    dst[(u0 + 1) ^ (r & 7)] = make_uint4(0u, 0u, 0u, 0u);
     return;
   }
   float v[64];
@@ -74,20 +98,16 @@ __global__ void __launch_bounds__(128) pack_kernel(PackParams p) {
     const float s_w = amax == 0.f ? 1.f : __fdiv_rn(amax, 2688.f);
     const float g_w = amax == 0.f ? 0.f : __fdiv_rn(448.f, amax);
     if (gid == 0) p.tensor_scale[0] = s_w;
-    const uint32_t s0 = quant_nv<32, false>(v, s_w, g_w, bytes, nullptr);
-    const uint32_t s1 = quant_nv<32, false>(v + 32, s_w, g_w, bytes + 16, nullptr);
-    *reinterpret_cast<uint16_t *>(p.sc_sparse + atom_offset(n, 2 * c, spr_sparse)) = (uint16_t)(s0 | (s1 << 8));
-    *reinterpret_cast<uint32_t *>(p.sc_dense + atom_offset(n, 4 * c, spr_dense)) =
-        s0 | (s0 << 8) | (s1 << 16) | (s1 << 24);
+    const uint32_t e0 = quant_nv<32, false>(v, s_w, g_w, bytes, nullptr);
+    const uint32_t e1 = quant_nv<32, false>(v + 32, s_w, g_w, bytes + 16, nullptr);
+    store_scales<FMT>(p, n, ks, s0, d0, e0 | (e1 << 8), e0 | (e0 << 8) | (e1 << 16) | (e1 << 24));
   } else {
     if (gid == 0) p.tensor_scale[0] = 1.f;
     const uint32_t e = quant_mx<64, false>(v, bytes, nullptr);
-    p.sc_sparse[atom_offset(n, c, spr_sparse)] = (uint8_t)e;
-    *reinterpret_cast<uint16_t *>(p.sc_dense + atom_offset(n, 2 * c, spr_dense)) = (uint16_t)(e | (e << 8));
+    store_scales<FMT>(p, n, ks, s0, d0, e, e | (e << 8));
   }
-  uint4 *dst = reinterpret_cast<uint4 *>(p.codes + (size_t)n * (p.K / 2) + (size_t)c * 32);
-  dst[0] = make_uint4(pack4(bytes), pack4(bytes + 4), pack4(bytes + 8), pack4(bytes + 12));
-  dst[1] = make_uint4(pack4(bytes + 16), pack4(bytes + 20), pack4(bytes + 24), pack4(bytes + 28));
+  dst[u0 ^ (r & 7)] = make_uint4(pack4(bytes), pack4(bytes + 4), pack4(bytes + 8), pack4(bytes + 12));
+  dst[(u0 + 1) ^ (r & 7)] = make_uint4(pack4(bytes + 16), pack4(bytes + 20), pack4(bytes + 24), pack4(bytes + 28));
 }
 
 }  // namespace

@@ -16,8 +16,9 @@
 //   so it is the max of the group maxima) -> backbone codes for every element with the
 //   backbone block scale; the kept bytes are stored, the dropped ones zeroed ->
 //   dequantized backbone -> residual r = xh - deq -> residual block scale and codes.
-// Blocks spanning lanes reduce with warp shuffles; scales and metadata are written as
-// bytes straight into their 128x4-atom / slab layouts. The RMSNorm weight is staged once
+// Blocks spanning lanes reduce with warp shuffles. Every output goes straight into the
+// tiled activation operand (chunks of 128 rows x 256 K holding swizzled codes, metadata
+// and 128x4 scale atoms: the GEMM's shared-memory image); rows T..T_pad-1 are zeroed. The RMSNorm weight is staged once
 // per block in shared memory as float32. Float32 arithmetic uses explicit
 // round-to-nearest scalar operations, so no contraction changes a rounding.
 #include "sharq_common.cuh"
@@ -149,17 +150,54 @@ __device__ __forceinline__ void deq8(uint32_t w, float dec, float s_x, float *o)
   }
 }
 
-// Byte offset of scale s of `row` in a 128x4-atom scale tensor: row part + scale part.
-__device__ __forceinline__ size_t atom_row_part(int row, int spr) {
-  return (size_t)(row >> 7) * (spr >> 2) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4;
+// Where double piece dp (16 K positions) of a row lands in the tiled operand: its chunk
+// (128-row block, 256-K step), the row inside the block and the piece inside the step.
+struct Spot {
+  uint8_t *chunk;
+  int r, j;
+};
+template <int FMT, int UNIT, bool DENSE>
+__device__ __forceinline__ Spot spot(const PrepParams &p, int row, int dp) {
+  constexpr ActTile L = act_tile(FMT, UNIT, !DENSE);
+  Spot s;
+  s.chunk = p.tiles + ((size_t)(row >> 7) * p.KS + (dp >> 4)) * L.bytes;
+  s.r = row & 127;
+  s.j = dp & 15;
+  return s;
 }
-__device__ __forceinline__ size_t atom_scale_part(int s) { return (size_t)(s >> 2) * 512 + (s & 3); }
+
+// Store the results of one double piece: backbone codes (4 bytes: 8 kept values), its
+// metadata (pair unit 8 bits, element unit 16 bits), the backbone block scale (written by
+// the first lane of its block), residual codes (8 bytes) and residual block scale.
+template <int FMT, int UNIT, bool DENSE>
+__device__ __forceinline__ void store16(const Spot &o, uint32_t kept, uint32_t meta, uint32_t sc_sp, uint32_t r0,
+                                        uint32_t r1, uint32_t sc_res) {
+  constexpr ActTile L = act_tile(FMT, UNIT, !DENSE);
+  const int r = o.r, j = o.j;
+  if (!DENSE) {
+    // 64-byte rows, 16-byte unit j/4 swizzled with row bits 1..2
+    *reinterpret_cast<uint32_t *>(o.chunk + L.sp + r * 64 + (((j >> 2) ^ ((r >> 1) & 3)) << 4) + (j & 3) * 4) = kept;
+    if (UNIT == 2) o.chunk[L.meta + r * 16 + j] = (uint8_t)meta;
+    else *reinterpret_cast<uint16_t *>(o.chunk + L.meta + (j >> 3) * 2048 + r * 16 + (j & 7) * 2) = (uint16_t)meta;
+    if (FMT == kFmtNV) {  // one backbone scale per 2 pieces
+      if ((j & 1) == 0) o.chunk[L.sf_sp + atom_pos(r, j >> 1)] = (uint8_t)sc_sp;
+    } else if ((j & 3) == 0) {  // one per 4 pieces
+      o.chunk[L.sf_sp + atom_pos(r, j >> 2)] = (uint8_t)sc_sp;
+    }
+  }
+  // 128-byte rows, 16-byte unit j/2 swizzled with row bits 0..2
+  *reinterpret_cast<uint2 *>(o.chunk + L.res + r * 128 + (((j >> 1) ^ (r & 7)) << 4) + (j & 1) * 8) =
+      make_uint2(r0, r1);
+  if (FMT == kFmtNV) o.chunk[L.sf_res + atom_pos(r, j)] = (uint8_t)sc_res;
+  else if ((j & 1) == 0) o.chunk[L.sf_res + atom_pos(r, j >> 1)] = (uint8_t)sc_res;
+}
 
 // ---------------------------------------------------------------- one double piece
 // 16 normalized values of double piece `dp` (lane-aligned: dp % 32 == lane).
 template <int FMT, int UNIT, bool DENSE>
 __device__ __forceinline__ void process16(const PrepParams &p, float *v, int row, int dp, bool live, float s_x,
-                                          float g_x, size_t sp_row, size_t res_row) {
+                                          float g_x) {
+  uint32_t kept = 0u, meta = 0u, sc_sp = 0u;
   if (!DENSE) {
     // ---- mask
     uint32_t nib[4];
@@ -185,21 +223,19 @@ __device__ __forceinline__ void process16(const PrepParams &p, float *v, int row
     // ---- backbone block amax: 16 stored (NVFP4) = 2 lanes, 32 stored (MXFP4) = 4 lanes
     gmax = fmaxf(gmax, __shfl_xor_sync(kFull, gmax, 1));
     if (FMT == kFmtMX) gmax = fmaxf(gmax, __shfl_xor_sync(kFull, gmax, 2));
-    uint32_t sc_code;
     float mult, dec;
     bool zero;
     if (FMT == kFmtNV) {
       const NvScale s = nv_scale(gmax, s_x, g_x);
-      sc_code = s.code; mult = s.inv; dec = s.dec; zero = s.zero;
+      sc_sp = s.code; mult = s.inv; dec = s.dec; zero = s.zero;
     } else {
       const MxScale s = mx_scale(gmax);
-      sc_code = s.code; mult = s.mult; dec = s.dec; zero = s.zero;
+      sc_sp = s.code; mult = s.mult; dec = s.dec; zero = s.zero;
     }
     // ---- backbone codes of all 16 values; keep the selected ones
     uint32_t w0, w1;
     codes16(v, mult, w0, w1);
     if (zero) { w0 = 0u; w1 = 0u; }
-    uint32_t kept, meta;
     if (UNIT == 2) {
       // group g = word g: byte j = pair j; kept bytes i0, i1
       const uint32_t n0 = nib[0], n1 = nib[1];
@@ -230,56 +266,25 @@ __device__ __forceinline__ void process16(const PrepParams &p, float *v, int row
     deq8<FMT>(w1, dec, s_x, dq + 8);
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __fsub_rn(v[i], dq[i]);
-    // ---- stores: backbone codes (4 bytes per lane), metadata and backbone scale bytes
-    if (live) {
-      *reinterpret_cast<uint32_t *>(p.sp_codes + (size_t)row * (p.K / 4) + (size_t)dp * 4) = kept;
-      if (UNIT == 2)  // 8 bits per lane, 16 lanes per 128-bit slab row
-        p.meta[((size_t)(dp >> 4) * p.T_pad + row) * 16 + (dp & 15)] = (uint8_t)meta;
-      else  // 16 bits per lane, 8 lanes per slab row
-        *reinterpret_cast<uint16_t *>(p.meta + ((size_t)(dp >> 3) * p.T_pad + row) * 16 + (dp & 7) * 2) =
-            (uint16_t)meta;
-      if (FMT == kFmtNV) {  // one backbone scale per 2 lanes
-        if ((dp & 1) == 0) p.sp_scales[sp_row + atom_scale_part(dp >> 1)] = (uint8_t)sc_code;
-      } else if ((dp & 3) == 0) {  // one per 4 lanes
-        p.sp_scales[sp_row + atom_scale_part(dp >> 2)] = (uint8_t)sc_code;
-      }
-    }
   }
   // ---- residual (or xh itself for the dense quantizer): dense blocks
   float am = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(v[i]));
-  uint32_t r0, r1;
+  uint32_t r0, r1, sc_res;
   if (FMT == kFmtNV) {  // block = this lane's 16 values
     const NvScale s = nv_scale(am, s_x, g_x);
     codes16(v, s.inv, r0, r1);
     if (s.zero) { r0 = 0u; r1 = 0u; }
-    if (live) p.res_scales[res_row + atom_scale_part(dp)] = (uint8_t)s.code;
+    sc_res = s.code;
   } else {  // block of 32 = 2 lanes
     am = fmaxf(am, __shfl_xor_sync(kFull, am, 1));
     const MxScale s = mx_scale(am);
     codes16(v, s.mult, r0, r1);
     if (s.zero) { r0 = 0u; r1 = 0u; }
-    if (live && (dp & 1) == 0) p.res_scales[res_row + atom_scale_part(dp >> 1)] = (uint8_t)s.code;
+    sc_res = s.code;
   }
-  if (live) *reinterpret_cast<uint2 *>(p.res_codes + (size_t)row * (p.K / 2) + (size_t)dp * 8) = make_uint2(r0, r1);
-}
-
-// Zero the scale and metadata bytes that double piece dp of a padding row (T..T_pad-1)
-// would carry.
-template <int FMT, int UNIT, bool DENSE>
-__device__ __forceinline__ void zero_pad16(const PrepParams &p, int row, int dp, size_t sp_row, size_t res_row) {
-  if (!DENSE) {
-    if (UNIT == 2) p.meta[((size_t)(dp >> 4) * p.T_pad + row) * 16 + (dp & 15)] = 0;
-    else *reinterpret_cast<uint16_t *>(p.meta + ((size_t)(dp >> 3) * p.T_pad + row) * 16 + (dp & 7) * 2) = 0;
-    if (FMT == kFmtNV) {
-      if ((dp & 1) == 0) p.sp_scales[sp_row + atom_scale_part(dp >> 1)] = 0;
-    } else if ((dp & 3) == 0) {
-      p.sp_scales[sp_row + atom_scale_part(dp >> 2)] = 0;
-    }
-  }
-  if (FMT == kFmtNV) p.res_scales[res_row + atom_scale_part(dp)] = 0;
-  else if ((dp & 1) == 0) p.res_scales[res_row + atom_scale_part(dp >> 1)] = 0;
+  if (live) store16<FMT, UNIT, DENSE>(spot<FMT, UNIT, DENSE>(p, row, dp), kept, meta, sc_sp, r0, r1, sc_res);
 }
 
 // ---------------------------------------------------------------- team reductions
@@ -381,8 +386,6 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   float s_x, g_x;
   row_scales(FMT, am, s_x, g_x);
 
-  const size_t sp_row = DENSE ? 0 : atom_row_part(row, p.n_sf_sp);
-  const size_t res_row = atom_row_part(row, p.n_sf_res);
   const bool pad_row = !live_row && row < p.T_pad;
 #pragma unroll
   for (int i = 0; i < kMaxDP; ++i) {
@@ -399,9 +402,9 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = 0.f;
       }
-      process16<FMT, UNIT, DENSE>(p, v, row, dp, live, s_x, g_x, sp_row, res_row);
+      process16<FMT, UNIT, DENSE>(p, v, row, dp, live, s_x, g_x);
     } else if (pad_row && dp < ndp_row) {
-      zero_pad16<FMT, UNIT, DENSE>(p, row, dp, sp_row, res_row);
+      store16<FMT, UNIT, DENSE>(spot<FMT, UNIT, DENSE>(p, row, dp), 0u, 0u, 0u, 0u, 0u, 0u);
     }
   }
   if (live_row && wt == 0 && lane == 0) p.row_scale[row] = s_x;
@@ -435,7 +438,7 @@ cudaError_t launch_n(const PrepParams &p, bool norm, cudaStream_t st) {
 int prep_team_warps(int k) { return (k / 16 + 32 * kMaxDP - 1) / (32 * kMaxDP); }
 
 cudaError_t launch_prep(PrepParams p, int fmt, int unit, bool norm, bool dense, cudaStream_t st) {
-  p.C = p.K / 16;
+  p.KS = p.K / 256;
   p.TS = prep_team_warps(p.K);
   if (p.TS > 8) return cudaErrorInvalidValue;  // k > 32768: outside the supported range
   if (dense) {

@@ -41,17 +41,37 @@
  * aligned pairs, i.e. 4 of 8 elements. sharq_prepare also computes the
  * element pattern (2, 4, 1).
  *
- * Scale layout ("128x4 atoms"). A scale tensor of R rows (R padded to a
- * multiple of 128; 256 for activations) and S scales per row (S a multiple of 4) is stored as atoms
- * of 512 bytes: atom (R/128 block rb, scale group sg = s/4) at byte offset
- * (rb * S/4 + sg) * 512, and inside it the scale of row r, index s at
- * (r%32)*16 + ((r%128)/32)*4 + s%4. This is the layout the tensor core's
- * scale-factor copy reads.
- *
  * Sparse metadata. One 4-bit entry per group, the two kept unit indices
- * (i0 < i1) as i0 | i1<<2, group g of a row at bits 4g..4g+3 of that row's
- * bit string. Stored in slabs of 128 bits per row: slab j holds groups
- * [32j, 32j+32) of every row, slab-major: byte offset (j * tokens_pad + row) * 16.
+ * (i0 < i1) as i0 | i1<<2; group g of a row at bits 4g..4g+3 of that row's bit
+ * string (per 256 K positions: 128 bits for pairs, 256 bits for elements).
+ *
+ * Tiled operands. Activations and weights are stored as the tensor-core GEMM reads
+ * them: chunks of 128 rows x 256 K positions, one contiguous chunk per (128-row block
+ * rb, K step ks = k/256), chunk-major: chunk (rb, ks) at byte (rb * k/256 + ks) * C,
+ * C the chunk size below. Inside a chunk, with r = row % 128:
+ *   - codes with row pitch P (128 bytes for 256 codes, 64 bytes for 128 kept codes):
+ *     byte b of row r's codes at r*P + ((b/16) XOR s(r))*16 + b%16, where the 16-byte
+ *     unit is swizzled with s(r) = r%8 (P = 128) or (r/2)%4 (P = 64);
+ *   - a scale run ("128x4 atoms"): scale s (0-based within the K step) of row r at
+ *     (s/4)*512 + (r%32)*16 + (r/32)*4 + s%4;
+ *   - metadata: row r's 16 bytes of bit string at r*16 (pairs); for elements, the two
+ *     16-byte halves at h*2048 + r*16.
+ * Rows past the tensor's end (up to the padded row count) are zero.
+ *
+ * Prepared activation chunk (sharq_prepare), B = 16 (NVFP4) or 32 (MXFP4):
+ *   residual codes  offset 0,      128 rows x 128 bytes (256 codes)
+ *   backbone codes  offset 16384,  128 rows x 64 bytes (the 128 kept codes, in K order)
+ *   metadata        offset 24576,  2048 bytes (pairs) or 4096 bytes (elements)
+ *   backbone scales then residual scales, scale runs of 128/B and 256/B scales per row
+ *   C = 29696 (NVFP4, pairs), 28672 (MXFP4, pairs), 31744 (NVFP4, elements),
+ *       30720 (MXFP4, elements); padded rows: tokens_pad = tokens rounded up to 256.
+ * Dense-quantized activation chunk (sharq_quantize_dense): codes at 0 (128 x 128 bytes),
+ *   scale run at 16384 (256/B scales per row); C = 18432 (NVFP4) or 17408 (MXFP4).
+ * Packed weight chunk, for 128 weight rows = one half of a 256-row block (n_out_pad =
+ *   n_out rounded up to 256): codes at 0 (128 x 128 bytes); then the sparse-view scales
+ *   (256/(2B) per row) and the dense-view scales (256/B per row) of ALL 256 rows of the
+ *   block, each as two scale runs (rows 0..127 of the block, then rows 128..255), so the
+ *   chunks of both halves carry the same scales; C = 22528 (NVFP4) or 19456 (MXFP4).
  */
 #ifndef SHARQ_H
 #define SHARQ_H
@@ -74,50 +94,40 @@ typedef enum {
 } sharq_status;
 
 /* The prepared activation of one call of sharq_prepare. Device buffers, caller-owned.
- *   sparse_codes  [tokens][k*nm_n/nm_m/2] bytes: kept values in K order, E2M1 pairs
- *   sparse_meta   metadata slabs (see above), k/(32*nm_m*unit) slabs of tokens_pad*16 bytes
- *   sparse_scales 128x4 atoms, tokens_pad rows, k*nm_n/nm_m/B scales per row; a backbone
- *                 block is B consecutive *stored* values (B = 16 NVFP4, 32 MXFP4)
- *   resid_codes   [tokens][k/2] bytes: the residual, E2M1 pairs
- *   resid_scales  128x4 atoms, tokens_pad rows, k/B scales per row
- *   row_scale     [tokens] float32: NVFP4 second-level scale s_x (1.0 for MXFP4)
- * tokens_pad = tokens rounded up to 256 (the GEMM's CTA pairs cover 256 rows). */
+ *   tiles      prepared activation chunks (see "Tiled operands"): backbone codes,
+ *              metadata and scales, residual codes and scales
+ *   row_scale  [tokens] float32: NVFP4 second-level scale s_x (1.0 for MXFP4) */
 typedef struct {
-  void *sparse_codes;
-  void *sparse_meta;
-  void *sparse_scales;
-  void *resid_codes;
-  void *resid_scales;
+  void *tiles;
   float *row_scale;
   int tokens, k, nm_n, nm_m, unit;
   int fmt; /* sharq_fmt */
 } sharq_prep;
 
 /* One packed weight [n_out][k]: a single E2M1 code payload and two scale views.
- *   codes          [n_out][k/2] bytes
- *   scales_sparse  128x4 atoms, n_out_pad rows, k/(2B) scales per row: one scale per 2B
- *                  consecutive K, the span of one backbone block at density 1/2
- *   scales_dense   128x4 atoms, n_out_pad rows, k/B scales per row: scales_sparse with
- *                  each entry repeated for the two B-wide dense blocks it covers
+ *   tiles          packed weight chunks (see "Tiled operands"): the codes, the sparse
+ *                  view (one scale per 2B consecutive K, the span of one backbone
+ *                  block at density 1/2) and the dense view (each sparse-view scale
+ *                  repeated for the two B-wide dense blocks it covers)
  *   tensor_scale   float32[2]: [0] = s_w (NVFP4 per-tensor scale, 1.0 for MXFP4),
- *                  [1] = amax|W| (written by sharq_pack_weight)
- * n_out_pad = n_out rounded up to 128. */
+ *                  [1] = amax|W| (written by sharq_pack_weight) */
 typedef struct {
-  void *codes;
-  void *scales_sparse;
-  void *scales_dense;
+  void *tiles;
   float *tensor_scale;
   int n_out, k;
   int fmt; /* sharq_fmt */
 } sharq_wpack;
 
-/* Byte sizes of the six sharq_prep buffers, in struct order, written to sizes[0..5];
+/* Byte sizes of the sharq_prep buffers (tiles, row_scale), written to sizes[0..1];
  * returns their sum, or 0 (with sharq_last_error set) for invalid arguments. */
 size_t sharq_prep_buffer_sizes(int tokens, int k, int nm_n, int nm_m, int unit, int fmt,
-                               size_t sizes[6]);
+                               size_t sizes[2]);
 
-/* Byte sizes of codes, scales_sparse, scales_dense, tensor_scale; returns the sum or 0. */
-size_t sharq_wpack_buffer_sizes(int n_out, int k, int fmt, size_t sizes[4]);
+/* Byte sizes of the dense quantizer's buffers (tiles, row_scale); returns the sum or 0. */
+size_t sharq_dense_buffer_sizes(int tokens, int k, int fmt, size_t sizes[2]);
+
+/* Byte sizes of the sharq_wpack buffers (tiles, tensor_scale); returns the sum or 0. */
+size_t sharq_wpack_buffer_sizes(int n_out, int k, int fmt, size_t sizes[2]);
 
 /* Pack a bf16 weight once (offline): per-tensor amax, block scales over 2B
  * consecutive K, E2M1 codes, and both scale views. The abstract: "The two paths
@@ -156,14 +166,12 @@ int sharq_linear(const sharq_prep *a, const sharq_wpack *w, void *y_dev, int out
 /* The library's own dense FP4 baseline (the README's "NVFP4: dense FP4 baseline"):
  * optional RMSNorm + dense block quantization of xh with the same row-scale rule
  * (one launch), and a dense FP4 GEMM against the weight's dense view (one launch).
- *   codes_dev [tokens][k/2]; scales_dev 128x4 atoms (tokens_pad rows, k/B per row);
- *   row_scale_dev [tokens] float32. */
+ *   tiles_dev      dense-quantized activation chunks (sharq_dense_buffer_sizes)
+ *   row_scale_dev  [tokens] float32 */
 int sharq_quantize_dense(const void *x_bf16_dev, int tokens, int k, const void *gamma_bf16_dev,
-                         float eps, int fmt, void *codes_dev, void *scales_dev,
-                         float *row_scale_dev, void *stream);
-int sharq_linear_dense(const void *codes_dev, const void *scales_dev, const float *row_scale_dev,
-                       int tokens, int k, const sharq_wpack *w, void *y_dev, int out_dtype,
-                       void *stream);
+                         float eps, int fmt, void *tiles_dev, float *row_scale_dev, void *stream);
+int sharq_linear_dense(const void *tiles_dev, const float *row_scale_dev, int tokens, int k,
+                       const sharq_wpack *w, void *y_dev, int out_dtype, void *stream);
 
 /* Synchronizes `stream`, then reports and clears the device-side status word that
  * bounded waits set when they give up: SHARQ_OK or SHARQ_ERR_TIMEOUT (or SHARQ_ERR_CUDA). */

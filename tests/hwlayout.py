@@ -1,69 +1,144 @@
-"""Readers that turn the library's hardware layouts back into the oracle's canonical arrays.
+"""Readers that turn the library's tiled operands back into the oracle's canonical arrays.
 
-Test infrastructure, written from the layout contract in include/sharq.h (not from
-the CUDA sources): E2M1 pairs with the lower K index in the low nibble, 128x4 scale
-atoms, metadata slabs of 128 bits per row.
+Test infrastructure, written from the layout contract in include/sharq.h ("Tiled
+operands"), not from the CUDA sources: chunks of 128 rows x 256 K, chunk-major
+[row block][K step]; E2M1 pairs with the lower K index in the low nibble; code rows
+with their 16-byte units swizzled by row bits; scale runs of 128x4 atoms; metadata
+bit strings of 16 bytes per row per 256 K (pairs) or two such halves (elements).
 """
 from __future__ import annotations
 
 import numpy as np
 import torch
 
+KSTEP = 256
+
 
 def to_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy()
 
 
-def unpack_e2m1(buf: np.ndarray, rows: int, n_codes: int) -> np.ndarray:
-    b = np.asarray(buf, dtype=np.uint8).reshape(-1)[: rows * n_codes // 2].reshape(rows, n_codes // 2)
-    out = np.empty((rows, n_codes), dtype=np.uint8)
-    out[:, 0::2] = b & 0xF
-    out[:, 1::2] = b >> 4
+def act_layout(block: int, unit: int, sparse: bool = True) -> dict:
+    """Byte offsets inside one activation chunk and the chunk size C (header table)."""
+    sf_sp, sf_res = 128 // block, 256 // block  # scales per row per K step
+    if not sparse:
+        return dict(res=0, sf_res=16384, bytes=_round1k(16384 + 128 * sf_res), spk_res=sf_res)
+    meta = 2048 if unit == 2 else 4096
+    off_sp = 24576 + meta
+    off_res = off_sp + 128 * sf_sp
+    return dict(res=0, sp=16384, meta=24576, sf_sp=off_sp, sf_res=off_res, bytes=_round1k(off_res + 128 * sf_res),
+                spk_sp=sf_sp, spk_res=sf_res)
+
+
+def w_layout(block: int) -> dict:
+    sf_sp, sf_res = 128 // block, 256 // block
+    return dict(b=0, sf_sp=16384, sf_res=16384 + 256 * sf_sp, bytes=16384 + 256 * (sf_sp + sf_res),
+                spk_sp=sf_sp, spk_res=sf_res)
+
+
+def _round1k(n: int) -> int:
+    return (n + 1023) // 1024 * 1024
+
+
+def _chunk_base(rows: np.ndarray, ks: np.ndarray, k: int, chunk: int) -> np.ndarray:
+    return ((rows // 128) * (k // KSTEP) + ks) * chunk
+
+
+def code_bytes(buf: np.ndarray, rows: int, k: int, chunk: int, off: int, pitch: int) -> np.ndarray:
+    """[rows, pitch * k/256] code bytes of a code region (pitch 128 or 64 bytes per K step)."""
+    b = np.asarray(buf, dtype=np.uint8).reshape(-1)
+    r = np.arange(rows)[:, None]
+    j = np.arange(pitch * (k // KSTEP))[None, :]  # byte index along the row
+    ks, within = j // pitch, j % pitch
+    rr = r % 128
+    swz = rr % 8 if pitch == 128 else (rr // 2) % 4
+    addr = _chunk_base(r, ks, k, chunk) + off + rr * pitch + ((within // 16) ^ swz) * 16 + within % 16
+    return b[addr]
+
+
+def nibbles(byts: np.ndarray) -> np.ndarray:
+    out = np.empty((byts.shape[0], 2 * byts.shape[1]), dtype=np.uint8)
+    out[:, 0::2] = byts & 0xF
+    out[:, 1::2] = byts >> 4
     return out
 
 
-def atom_index(rows: int, spr: int) -> np.ndarray:
-    """Byte offset of every (row, scale) in a 128x4-atom scale tensor: [rows, spr]."""
-    r = np.arange(rows)[:, None]
-    s = np.arange(spr)[None, :]
-    return ((r // 128) * (spr // 4) + s // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + s % 4
+def scale_run(buf: np.ndarray, rows: int, k: int, chunk: int, off: int, spk: int, row_of=None) -> np.ndarray:
+    """[rows, spk * k/256] scale bytes of a scale run (spk scales per row per K step).
 
-
-def unswizzle_scales(buf: np.ndarray, rows: int, spr: int) -> np.ndarray:
-    return np.asarray(buf, dtype=np.uint8).reshape(-1)[atom_index(rows, spr)]
-
-
-def meta_to_idx(buf: np.ndarray, tokens: int, k: int, unit: int) -> np.ndarray:
-    """Kept unit indices [tokens, G, 2] from metadata slabs (groups of 4 units)."""
-    tp = (tokens + 255) // 256 * 256
-    G = k // (4 * unit)
+    row_of maps a row to (chunk row for the chunk base, row inside the run's 128-row
+    atoms, extra byte offset) for the weight's 256-row-block runs."""
     b = np.asarray(buf, dtype=np.uint8).reshape(-1)
-    g = np.arange(G)
+    r = np.arange(rows)[:, None]
+    s = np.arange(spk * (k // KSTEP))[None, :]
+    ks, sl = s // spk, s % spk
+    if row_of is None:
+        base_row, rr, extra = r, r % 128, 0
+    else:
+        base_row, rr, extra = row_of(r)
+    addr = (_chunk_base(base_row, ks, k, chunk) + off + extra + (sl // 4) * 512 + (rr % 32) * 16 + (rr // 32) * 4
+            + sl % 4)
+    return b[addr]
+
+
+def meta_idx(buf: np.ndarray, tokens: int, k: int, unit: int, chunk: int, off: int) -> np.ndarray:
+    """Kept unit indices [tokens, G, 2] (groups of 4 units) from the metadata bit strings."""
+    b = np.asarray(buf, dtype=np.uint8).reshape(-1)
+    per_step = KSTEP // (4 * unit)  # groups per K step: 32 (pairs) or 64 (elements)
+    g = np.arange(k // (4 * unit))[None, :]
     t = np.arange(tokens)[:, None]
-    byte = ((g // 32)[None, :] * tp + t) * 16 + (g % 32)[None, :] // 2
-    nib = (b[byte] >> (4 * (g % 2))[None, :]) & 0xF
+    ks, gg = g // per_step, g % per_step
+    half, gh = gg // 32, gg % 32
+    addr = _chunk_base(t, ks, k, chunk) + off + half * 2048 + (t % 128) * 16 + gh // 2
+    nib = (b[addr] >> (4 * (gh % 2))) & 0xF
     return np.stack([nib & 3, nib >> 2], axis=-1).astype(np.int64)
 
 
 def read_prep(p, block: int) -> dict:
     """Canonical arrays of a library Prep (pattern 2:4) for comparison with oracle.prepare."""
     T, K, unit = p.tokens, p.k, p.unit
-    stored = K // 2
+    L = act_layout(block, unit)
+    buf = to_np(p.tiles)
     return dict(
-        idx=meta_to_idx(to_np(p.sparse_meta), T, K, unit),
-        sp_codes=unpack_e2m1(to_np(p.sparse_codes), T, stored),
-        sp_scales=unswizzle_scales(to_np(p.sparse_scales), T, stored // block),
-        res_codes=unpack_e2m1(to_np(p.resid_codes), T, K),
-        res_scales=unswizzle_scales(to_np(p.resid_scales), T, K // block),
+        idx=meta_idx(buf, T, K, unit, L["bytes"], L["meta"]),
+        sp_codes=nibbles(code_bytes(buf, T, K, L["bytes"], L["sp"], 64)),
+        sp_scales=scale_run(buf, T, K, L["bytes"], L["sf_sp"], L["spk_sp"]),
+        res_codes=nibbles(code_bytes(buf, T, K, L["bytes"], L["res"], 128)),
+        res_scales=scale_run(buf, T, K, L["bytes"], L["sf_res"], L["spk_res"]),
         row_scale=to_np(p.row_scale),
     )
 
 
-def read_wpack(w, block: int) -> dict:
+def read_dense(q, block: int) -> dict:
+    """Codes and scales of a dense-quantized activation (sharq_quantize_dense)."""
+    T, K = q.tokens, q.k
+    L = act_layout(block, 2, sparse=False)
+    buf = to_np(q.tiles)
+    return dict(codes=nibbles(code_bytes(buf, T, K, L["bytes"], L["res"], 128)),
+                scales=scale_run(buf, T, K, L["bytes"], L["sf_res"], L["spk_res"]),
+                row_scale=to_np(q.row_scale))
+
+
+def read_wpack(w, block: int, half: str = "own") -> dict:
+    """Canonical arrays of a packed weight. `half` picks which copy of the block's scales
+    is read: "own" (the chunk of the row's half), "lo" or "hi" (the block's first or second
+    half chunk)."""
     N, K = w.n_out, w.k
+    L = w_layout(block)
+    buf = to_np(w.tiles)
+
+    def run(off, spk):
+        def row_of(r):
+            blk_half = (r // 128) % 2
+            pick = {"own": blk_half, "lo": np.zeros_like(blk_half), "hi": np.ones_like(blk_half)}[half]
+            base_row = (r // 256) * 256 + pick * 128
+            extra = blk_half * 128 * spk  # second run of the block for its upper 128 rows
+            return base_row, r % 128, extra
+        return scale_run(buf, N, K, L["bytes"], off, spk, row_of)
+
     return dict(
-        codes=unpack_e2m1(to_np(w.codes), N, K),
-        scales_sparse=unswizzle_scales(to_np(w.scales_sparse), N, K // (2 * block)),
-        scales_dense=unswizzle_scales(to_np(w.scales_dense), N, K // block),
+        codes=nibbles(code_bytes(buf, N, K, L["bytes"], L["b"], 128)),
+        scales_sparse=run(L["sf_sp"], L["spk_sp"]),
+        scales_dense=run(L["sf_res"], L["spk_res"]),
         tensor_scale=to_np(w.tensor_scale)[0],
     )

@@ -34,23 +34,24 @@ def test_exports_every_declared_symbol(S):
 
 
 def test_version(S):
-    assert S.lib.sharq_version() == 100
+    assert S.lib.sharq_version() == 200
 
 
 def test_prep_buffer_sizes(S):
+    """Chunks of 128 rows x 256 K over tokens padded to 256, sizes from the header's table."""
     T, K = 300, 4096
-    s = S.sharq_prep_buffer_sizes(T, K, 2, 4, 2, "nvfp4")
-    Tp = 512
-    assert s == [T * K // 4, (K // 256) * Tp * 16, Tp * K // 32, T * K // 2, Tp * K // 16, T * 4]
-    s = S.sharq_prep_buffer_sizes(T, K, 2, 4, 1, "mxfp4")
-    assert s == [T * K // 4, (K // 128) * Tp * 16, Tp * K // 64, T * K // 2, Tp * K // 32, T * 4]
+    chunks = (512 // 128) * (K // 256)
+    assert S.sharq_prep_buffer_sizes(T, K, 2, 4, 2, "nvfp4") == [chunks * 29696, T * 4]
+    assert S.sharq_prep_buffer_sizes(T, K, 2, 4, 2, "mxfp4") == [chunks * 28672, T * 4]
+    assert S.sharq_prep_buffer_sizes(T, K, 2, 4, 1, "nvfp4") == [chunks * 31744, T * 4]
+    assert S.sharq_prep_buffer_sizes(T, K, 2, 4, 1, "mxfp4") == [chunks * 30720, T * 4]
+    assert S.sharq_dense_buffer_sizes(T, K, "nvfp4") == [chunks * 18432, T * 4]
+    assert S.sharq_dense_buffer_sizes(T, K, "mxfp4") == [chunks * 17408, T * 4]
 
 
 def test_wpack_buffer_sizes(S):
-    s = S.sharq_wpack_buffer_sizes(6144, 4096, "nvfp4")
-    assert s == [6144 * 2048, 6144 * 4096 // 32, 6144 * 4096 // 16, 8]
-    s = S.sharq_wpack_buffer_sizes(208, 256, "mxfp4")
-    assert s == [208 * 128, 256 * 4, 256 * 8, 8]
+    assert S.sharq_wpack_buffer_sizes(6144, 4096, "nvfp4") == [(6144 // 128) * 16 * 22528, 8]
+    assert S.sharq_wpack_buffer_sizes(208, 256, "mxfp4") == [(256 // 128) * 1 * 19456, 8]
 
 
 @pytest.mark.parametrize("args,status", [
@@ -62,7 +63,7 @@ def test_wpack_buffer_sizes(S):
     ((16, 4096, 4, 8, 1, 0), 2),    # valid pattern this build does not execute
 ])
 def test_prep_sizes_reject(S, args, status):
-    sizes = (ctypes.c_size_t * 6)()
+    sizes = (ctypes.c_size_t * 2)()
     assert S.lib.sharq_prep_buffer_sizes(*args, sizes) == 0
     assert S.last_error()
 
@@ -85,8 +86,8 @@ def test_calls_reject_bad_arguments_before_launch(S):
     # weight pack: bad n_out
     assert S.lib.sharq_pack_weight(ctypes.c_void_p(0x1000), 20, 4096, 0, ctypes.byref(W), null) == S.SHARQ_ERR_INVALID_ARG
     # linear: mismatched formats / k / element pattern
-    P2 = S._Prep(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 16, 4096, 2, 4, 2, 0)
-    W2 = S._WPack(0x1000, 0x1000, 0x1000, 0x1000, 256, 4096, 1)
+    P2 = S._Prep(0x1000, 0x1000, 16, 4096, 2, 4, 2, 0)
+    W2 = S._WPack(0x1000, 0x1000, 256, 4096, 1)
     assert S.lib.sharq_linear(ctypes.byref(P2), ctypes.byref(W2), ctypes.c_void_p(0x1000), 0, null) == S.SHARQ_ERR_INVALID_ARG
     assert "format mismatch" in S.last_error()
     W2.fmt, W2.k = 0, 2048
@@ -96,4 +97,4 @@ def test_calls_reject_bad_arguments_before_launch(S):
     assert S.lib.sharq_linear(ctypes.byref(P2), None, ctypes.c_void_p(0x1000), 0, null) == S.SHARQ_ERR_INVALID_ARG
     P2.unit = 2
     assert S.lib.sharq_linear(ctypes.byref(P2), ctypes.byref(W2), ctypes.c_void_p(0x1000), 5, null) == S.SHARQ_ERR_INVALID_ARG
-    assert S.lib.sharq_linear_dense(None, None, None, 16, 4096, ctypes.byref(W2), None, 0, null) == S.SHARQ_ERR_INVALID_ARG
+    assert S.lib.sharq_linear_dense(None, None, 16, 4096, ctypes.byref(W2), None, 0, null) == S.SHARQ_ERR_INVALID_ARG

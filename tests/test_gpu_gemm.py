@@ -27,11 +27,17 @@ def test_pack_weight_bit_exact(fmt, N, K):
     w = to_dev_bf16(w_bits)
     wp = S.sharq_pack_weight(w, fmt)
     torch.cuda.synchronize()
-    got = hw.read_wpack(wp, O.block_size(FMT_NAME[fmt]))
+    B = O.block_size(FMT_NAME[fmt])
+    got = hw.read_wpack(wp, B)
     ref = O.pack_weight(f32(w_bits), FMT_NAME[fmt])
     for key in ("codes", "scales_sparse", "scales_dense"):
         assert np.array_equal(got[key], ref[key]), key
     assert got["tensor_scale"] == ref["tensor_scale"]
+    # both halves of a 256-row block carry the block's scales
+    for half in ("lo", "hi"):
+        cp = hw.read_wpack(wp, B, half)
+        assert np.array_equal(cp["scales_sparse"], ref["scales_sparse"]), half
+        assert np.array_equal(cp["scales_dense"], ref["scales_dense"]), half
 
 
 def run_linear(S, x_bits, w_bits, fmt, out_dtype=torch.float32):

@@ -125,9 +125,10 @@ def test_dense_quantizer_matches_oracle(fmt):
     B = O.block_size(FMT_NAME[fmt])
     T, K = lin.x.shape
     ref = O.quantize_dense(f32(lin.x), None, lin.eps, FMT_NAME[fmt])
-    assert np.array_equal(hw.unpack_e2m1(hw.to_np(q.codes), T, K), ref["codes"])
-    assert np.array_equal(hw.unswizzle_scales(hw.to_np(q.scales), T, K // B), ref["scales"])
-    assert np.array_equal(hw.to_np(q.row_scale), ref["row_scale"])
+    got = hw.read_dense(q, B)
+    assert np.array_equal(got["codes"], ref["codes"])
+    assert np.array_equal(got["scales"], ref["scales"])
+    assert np.array_equal(got["row_scale"], ref["row_scale"])
 
 
 @pytest.mark.parametrize("which,T", [("qkv", 2048), ("down", 4096), ("qwen_down", 300), ("qwen_qkv", 130)])
