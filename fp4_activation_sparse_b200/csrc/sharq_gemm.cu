@@ -18,13 +18,17 @@
 //   warp 0      TMA producer (both CTAs): the activation chunk and the weight chunk of the
 //               K step; every load completes on the leader CTA's barrier.
 //   warp 1      TMEM owner (both CTAs) and, in the leader, the single MMA-issuing thread:
-//               tcgen05.cp moves scales and metadata to tensor memory, then two
-//               tcgen05.mma.sp (K=128 logical, pairwise 4:8) and four dense tcgen05.mma
-//               (K=64) accumulate into one fp32 accumulator of 128 x 256 per CTA. Both
-//               paths carry the same per-row scale s_x, so one accumulator holds their sum.
-//               Each weight chunk feeds both MMAs. Commits arrive on both CTAs' barriers
-//               (multicast commit).
-//   warps 2..9  epilogue (both CTAs): tcgen05.ld, y = acc * s_x[row] * s_w, bf16/fp32 stores.
+//               two tcgen05.mma.sp (K=128 logical, pairwise 4:8) and four dense tcgen05.mma
+//               (K=64) per K step accumulate into one fp32 accumulator of 128 x 256 per CTA.
+//               Both paths carry the same per-row scale s_x, so one accumulator holds their
+//               sum. Each weight chunk feeds both MMAs. Commits arrive on both CTAs'
+//               barriers (multicast commit).
+//   warp 10     scale copier (leader): tcgen05.cp of the K step's scales and metadata into
+//               one of two tensor-memory buffers, from its own thread so that the copies of
+//               step k+1 are issued while the MMAs of step k run.
+//   warps 2..9  epilogue (both CTAs): tcgen05.ld of the whole accumulator into registers, release
+//               of the tensor memory, then y = acc * s_x[row] * s_w as bf16/fp32 stores while the
+//               next tile's MMAs run.
 // Every mbarrier wait is bounded by a time limit; on expiry the CTA records a status word,
 // stops issuing, drains (bounded) what it issued, frees TMEM and exits.
 #include <cuda.h>
@@ -46,7 +50,7 @@ constexpr int BN = 256;   // output columns per pair tile
 constexpr int BK = 256;   // logical K per stage
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kThreads = 64 + 32 * kEpiWarps + 32;  // producer, MMA, epilogue, scale copier
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = 256;
 constexpr uint32_t kScaleBufCols = 80;  // per K-tile parity: meta 4, SFA_sp 8, SFA_res 16, SFB_sp 16, SFB_res 32
@@ -171,6 +175,15 @@ __device__ __forceinline__ void tc_commit_both(uint32_t bar) {
       : "memory");
 }
 
+// arrive once on the leader CTA's barrier at this offset when this thread's tcgen05 operations finish
+__device__ __forceinline__ void tc_commit_leader(uint32_t bar) {
+  const uint16_t mask = 0x1;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
 // Shared-memory matrix descriptors (K-major) as templates with the address field zero;
 // layout 0 none, 2 SW128, 4 SW64; bit 46 is the sm_100 descriptor version. dsc() adds the
 // 16-byte-unit address of one operand.
@@ -242,7 +255,8 @@ __device__ __forceinline__ void tc_cp_128x128(uint32_t taddr, uint64_t desc) {
   asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
+// 32 lanes x 32 columns of 32 bits; asynchronous until tmem_ld_wait()
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t *r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
       "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
@@ -251,7 +265,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
         "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Orders every later use of r after the preceding tmem_ld_wait(): the registers written by
+// an asynchronous tensor-memory load are only valid once the wait has returned.
+__device__ __forceinline__ void reg_fence32(uint32_t *r) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 }
 
 template <bool MX, bool SPARSE>
@@ -260,8 +286,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kMaxStageBytes);
-  // bars: full[kStages], empty[kStages], acc_full, acc_empty, drain
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kStages + 3);
+  // bars: full[kStages], empty[kStages], acc_full, acc_empty, drain, sf_full[kStages], sf_free[2], sf_drain
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 6);
   volatile uint32_t *abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -272,6 +298,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
   const uint32_t acc_full = bar0 + 8u * (2 * kStages), acc_empty = acc_full + 8, drain_bar = acc_full + 16;
+  auto sf_full_bar = [&](int s) { return bar0 + 8u * (2 * kStages + 3 + s); };
+  auto sf_free_bar = [&](int b) { return bar0 + 8u * (3 * kStages + 3 + b); };
+  const uint32_t sf_drain_bar = bar0 + 8u * (3 * kStages + 5);
 
   using L = Stage<MX, SPARSE>;
   constexpr int apt_res = atoms_res(MX ? 1 : 0), apt_sp = atoms_sp(MX ? 1 : 0);
@@ -289,6 +318,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kEpiWarps);
     mbar_init(drain_bar, 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(sf_full_bar(s), 1);
+    mbar_init(sf_free_bar(0), 1);
+    mbar_init(sf_free_bar(1), 1);
+    mbar_init(sf_drain_bar, 1);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -352,38 +385,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer (leader CTA)
     if (lane == 0 && leader) {
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      uint32_t phase = 0, acc_phase = 0, step = 0;
       bool ok = true;
       const uint32_t acc = tmem;  // lanes 0..127 of each CTA, columns 0..255
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
         if (!mbar_wait(acc_empty, acc_phase ^ 1u, limit, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        for (int kt = 0; kt < num_k; ++kt) {
+        for (int kt = 0; kt < num_k; ++kt, ++step) {
+          // the scale copier waited for this stage's bytes before copying its scales
+          if (!mbar_wait(sf_full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
           if (!mbar_wait(full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
           tc_fence_after();
           // descriptors: constant templates plus the operand's shared-memory address >> 4
           const uint32_t st4 = (smem0 + stage * kStageBytes) >> 4;
-          const uint32_t sbuf = tmem + kAccCols + (kt & 1) * kScaleBufCols;
+          const uint32_t sbuf = tmem + kAccCols + (step & 1u) * kScaleBufCols;
           const uint32_t t_meta = sbuf, t_sfa_sp = sbuf + 4, t_sfa_res = sbuf + 12, t_sfb_sp = sbuf + 28,
                          t_sfb_res = sbuf + 44;
           constexpr int kA = 0, kW = L::kW;
-          // scales and metadata: shared memory -> tensor memory (both CTAs). The weight
-          // chunk holds the scales of both 128-row halves of the pair's 256 columns.
-#pragma unroll
-          for (int a = 0; a < apt_res; ++a) {
-            tc_cp_atom(t_sfa_res + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_res + a * 512) / 16));
-            tc_cp_atom(t_sfb_res + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_res + a * 512) / 16));
-            tc_cp_atom(t_sfb_res + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_res + (apt_res + a) * 512) / 16));
-          }
-          if (SPARSE) {
-            tc_cp_128x128(t_meta, dsc(kDescNone, st4 + (kA + L::A.meta) / 16));
-#pragma unroll
-            for (int a = 0; a < apt_sp; ++a) {
-              tc_cp_atom(t_sfa_sp + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_sp + a * 512) / 16));
-              tc_cp_atom(t_sfb_sp + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_sp + a * 512) / 16));
-              tc_cp_atom(t_sfb_sp + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_sp + (apt_sp + a) * 512) / 16));
-            }
-          }
           uint32_t accumulate = kt > 0 ? 1u : 0u;
           if (SPARSE) {
             // two sparse MMAs: 128 logical K each = 32 bytes of compressed A, 64 bytes of B
@@ -409,6 +427,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             accumulate = 1u;
           }
           tc_commit_both(empty_bar(stage));  // frees the stage in both CTAs once these MMAs have read it
+          tc_commit_leader(sf_free_bar(step & 1u));  // and the scale buffer
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -420,7 +439,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       volatile uint32_t no_abort = 0;
       mbar_wait(drain_bar, 0, kDrainLimitNs, &no_abort);
     }
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     // ------------------------------------------------------------ epilogue (warps 2..9, both CTAs)
     const int quarter = warp & 3;          // TMEM lane quarter this warp may access
     const int col_half = (warp - 2) >> 2;  // columns [128*col_half, 128*col_half + 128)
@@ -430,53 +449,104 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const float s_w = p.tensor_scale[0];
     for (int tile = pair; tile < num_tiles; tile += num_pairs) {
       const int m0 = (tile % num_m) * (2 * BM) + (int)rank * BM, n0 = (tile / num_m) * BN;
-      if (!mbar_wait(acc_full, acc_phase, limit, abort_flag)) break;
-      tc_fence_after();
       const int row = m0 + r_local;
       const float scale = row < p.T ? __fmul_rn(p.row_scale[row], s_w) : 0.f;
-      for (int c0 = col_half * 128; c0 < col_half * 128 + 128; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + c0, r);
-        const int col = n0 + c0;
-        if (row < p.T && col < p.N) {
-          if (p.out_f32) {
-            float *dst = reinterpret_cast<float *>(p.y) + (size_t)row * p.N + col;
-            if (col + 32 <= p.N) {
+      if (!mbar_wait(acc_full, acc_phase, limit, abort_flag)) break;
+      tc_fence_after();
+      // Read this warp's 32 rows x 128 columns of the accumulator, then hand the tensor memory
+      // back at once: the stores below overlap the next tile's MMAs.
+      uint32_t r[4][32];
 #pragma unroll
-              for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4 *>(dst + i) =
-                    make_float4(__fmul_rn(__uint_as_float(r[i]), scale), __fmul_rn(__uint_as_float(r[i + 1]), scale),
-                                __fmul_rn(__uint_as_float(r[i + 2]), scale), __fmul_rn(__uint_as_float(r[i + 3]), scale));
-            } else {
+      for (int c = 0; c < 4; ++c) tmem_ld32_async(tmem + ((uint32_t)(quarter * 32) << 16) + col_half * 128 + 32 * c, r[c]);
+      tmem_ld_wait();
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (col + i < p.N) dst[i] = __fmul_rn(__uint_as_float(r[i]), scale);
-            }
-          } else {
-            uint32_t packed[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * i]), scale),
-                                                             __fmul_rn(__uint_as_float(r[2 * i + 1]), scale));
-              packed[i] = *reinterpret_cast<const uint32_t *>(&h);
-            }
-            uint16_t *dst = reinterpret_cast<uint16_t *>(p.y) + (size_t)row * p.N + col;
-            if (col + 32 <= p.N) {
-#pragma unroll
-              for (int i = 0; i < 16; i += 4)
-                *reinterpret_cast<uint4 *>(dst + 2 * i) = make_uint4(packed[i], packed[i + 1], packed[i + 2], packed[i + 3]);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                if (col + 2 * i < p.N) *reinterpret_cast<uint32_t *>(dst + 2 * i) = packed[i];
-            }
-          }
-        }
-      }
+      for (int c = 0; c < 4; ++c) reg_fence32(r[c]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
       acc_phase ^= 1u;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int col = n0 + col_half * 128 + 32 * c;
+        if (row >= p.T || col >= p.N) continue;
+        if (p.out_f32) {
+          float *dst = reinterpret_cast<float *>(p.y) + (size_t)row * p.N + col;
+          if (col + 32 <= p.N) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4 *>(dst + i) = make_float4(
+                  __fmul_rn(__uint_as_float(r[c][i]), scale), __fmul_rn(__uint_as_float(r[c][i + 1]), scale),
+                  __fmul_rn(__uint_as_float(r[c][i + 2]), scale), __fmul_rn(__uint_as_float(r[c][i + 3]), scale));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (col + i < p.N) dst[i] = __fmul_rn(__uint_as_float(r[c][i]), scale);
+          }
+        } else {
+          uint32_t packed[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[c][2 * i]), scale),
+                                                           __fmul_rn(__uint_as_float(r[c][2 * i + 1]), scale));
+            packed[i] = *reinterpret_cast<const uint32_t *>(&h);
+          }
+          uint16_t *dst = reinterpret_cast<uint16_t *>(p.y) + (size_t)row * p.N + col;
+          if (col + 32 <= p.N) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+              *reinterpret_cast<uint4 *>(dst + 2 * i) = make_uint4(packed[i], packed[i + 1], packed[i + 2], packed[i + 3]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (col + 2 * i < p.N) *reinterpret_cast<uint32_t *>(dst + 2 * i) = packed[i];
+          }
+        }
+      }
+    }
+  }
+
+  else {
+    // ------------------------------------------------------------ scale copier (warp 10, leader)
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0, step = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        for (int kt = 0; kt < num_k; ++kt, ++step) {
+          if (!mbar_wait(full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
+          // buffer step%2 is free once the MMAs of step-2 completed
+          if (!mbar_wait(sf_free_bar(step & 1u), ((step >> 1) & 1u) ^ 1u, limit, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t st4 = (smem0 + stage * kStageBytes) >> 4;
+          const uint32_t sbuf = tmem + kAccCols + (step & 1u) * kScaleBufCols;
+          const uint32_t t_meta = sbuf, t_sfa_sp = sbuf + 4, t_sfa_res = sbuf + 12, t_sfb_sp = sbuf + 28,
+                         t_sfb_res = sbuf + 44;
+          constexpr int kA = 0, kW = L::kW;
+          // shared memory -> tensor memory (both CTAs). The weight chunk holds the scales of
+          // both 128-row halves of the pair's 256 columns.
+#pragma unroll
+          for (int a = 0; a < apt_res; ++a) {
+            tc_cp_atom(t_sfa_res + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_res + a * 512) / 16));
+            tc_cp_atom(t_sfb_res + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_res + a * 512) / 16));
+            tc_cp_atom(t_sfb_res + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_res + (apt_res + a) * 512) / 16));
+          }
+          if (SPARSE) {
+            tc_cp_128x128(t_meta, dsc(kDescNone, st4 + (kA + L::A.meta) / 16));
+#pragma unroll
+            for (int a = 0; a < apt_sp; ++a) {
+              tc_cp_atom(t_sfa_sp + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_sp + a * 512) / 16));
+              tc_cp_atom(t_sfb_sp + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_sp + a * 512) / 16));
+              tc_cp_atom(t_sfb_sp + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_sp + (apt_sp + a) * 512) / 16));
+            }
+          }
+          tc_commit_leader(sf_full_bar(stage));
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Drain: the copies issued above complete before TMEM is released.
+      tc_commit_leader(sf_drain_bar);
+      volatile uint32_t no_abort = 0;
+      mbar_wait(sf_drain_bar, 0, kDrainLimitNs, &no_abort);
     }
   }
 
