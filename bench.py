@@ -202,15 +202,32 @@ def run_sharq(args, rank, world, local):
     del w_dev
     stream = torch.cuda.current_stream()
 
-    def step(i):
+    def step(i, st):
         s = i % nsets
-        S.sharq_prepare(xs[s], gamma, lin.eps, 2, 4, 2, "nvfp4", out=preps[s], stream=stream)
-        S.sharq_linear(preps[s], wps[s], y=ys[s], stream=stream)
+        S.sharq_prepare(xs[s], gamma, lin.eps, 2, 4, 2, "nvfp4", out=preps[s], stream=st)
+        S.sharq_linear(preps[s], wps[s], y=ys[s], stream=st)
 
     for i in range(args.warmup):
-        step(i)
+        step(i, stream)
     torch.cuda.synchronize()
     assert S.sharq_device_status() == S.SHARQ_OK
+
+    # ---- CUDA graphs: one per input set for the whole step (prepare + linear), and per kernel
+    # over all sets, so that the device-timed loops replay launches without Python/ctypes
+    # overhead between them (a step is tens of microseconds of GPU time)
+    cap = torch.cuda.Stream()
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            fn(cap)
+        return g
+
+    step_graphs = [capture(lambda st, s=s: step(s, st)) for s in range(nsets)]
+    prep_graph = capture(lambda st: [S.sharq_prepare(xs[s], gamma, lin.eps, 2, 4, 2, "nvfp4", out=preps[s], stream=st)
+                                     for s in range(nsets)])
+    lin_graph = capture(lambda st: [S.sharq_linear(preps[s], wps[s], y=ys[s], stream=st) for s in range(nsets)])
+    torch.cuda.synchronize()
 
     # ---- device-timed whole steps; the clock sampler runs from a 1 s pre-roll of the same
     # step (nvidia-smi needs ~100 ms per sample) through the timed region
@@ -219,7 +236,7 @@ def run_sharq(args, rank, world, local):
         t_end = time.perf_counter() + 1.0
         i = 0
         while time.perf_counter() < t_end:
-            step(i)
+            step_graphs[i % nsets].replay()
             i += 1
             if i % 64 == 0:
                 torch.cuda.synchronize()
@@ -227,50 +244,40 @@ def run_sharq(args, rank, world, local):
         torch.cuda.synchronize()
         ev0.record(stream)
         for i in range(args.steps):
-            step(i)
+            step_graphs[i % nsets].replay()
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
     clocks = clk.summary()
+    assert S.sharq_device_status() == S.SHARQ_OK
 
-    # ---- per-kernel times (events around each launch on the launching stream)
-    def per_kernel(n):
-        tp, tl = [], []
-        for i in range(n):
-            s = i % nsets
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-            e[0].record(stream)
-            S.sharq_prepare(xs[s], gamma, lin.eps, 2, 4, 2, "nvfp4", out=preps[s], stream=stream)
-            e[1].record(stream)
-            S.sharq_linear(preps[s], wps[s], y=ys[s], stream=stream)
-            e[2].record(stream)
-            e[2].synchronize()
-            tp.append(e[0].elapsed_time(e[1]))
-            tl.append(e[1].elapsed_time(e[2]))
-        return statistics.median(tp), statistics.median(tl)
+    # ---- per-kernel times: each kernel alone, all input sets back to back (events on the
+    # launching stream around graph replays)
+    def graph_time(g, launches, reps=20):
+        for _ in range(3):
+            g.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b) / (reps * launches)
 
-    t_prep_ms, t_lin_ms = per_kernel(max(args.steps, 10))
+    t_prep_ms = graph_time(prep_graph, nsets)
+    t_lin_ms = graph_time(lin_graph, nsets)
 
     # ---- baselines on the same shapes: torch bf16 matmul and the library's dense NVFP4 pipeline
     q = S.sharq_quantize_dense(xs[0], gamma, lin.eps, "nvfp4")
     yd = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
     w_bf16 = to_dev(lin.w)
-
-    def timeit(f, n=20):
-        for _ in range(3):
-            f()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(n):
-            f()
-        b.record(stream)
-        b.synchronize()
-        return a.elapsed_time(b) / n
-
-    t_bf16 = timeit(lambda: torch.matmul(xs[0], w_bf16.t()))
-    t_dq = timeit(lambda: S.sharq_quantize_dense(xs[0], gamma, lin.eps, "nvfp4", out=q, stream=stream))
-    t_dl = timeit(lambda: S.sharq_linear_dense(q, wps[0], y=yd, stream=stream))
+    with torch.cuda.stream(cap):  # cuBLAS creates its handle and workspace outside the capture
+        torch.matmul(xs[0], w_bf16.t())
+    torch.cuda.synchronize()
+    t_bf16 = graph_time(capture(lambda st: torch.matmul(xs[0], w_bf16.t())), 1)
+    t_dq = graph_time(capture(lambda st: S.sharq_quantize_dense(xs[0], gamma, lin.eps, "nvfp4", out=q, stream=st)), 1)
+    t_dl = graph_time(capture(lambda st: S.sharq_linear_dense(q, wps[0], y=yd, stream=st)), 1)
     del w_bf16
 
     # ---- end to end through the public API with host buffers: every step copies its input
@@ -341,7 +348,8 @@ def run_sharq(args, rank, world, local):
         "data": "synthetic (seeded outlier-channel activations, N(0,0.02) weight)",
         "config": {"workload": f"llama31_8b_qkv_prefill T={T} K={K} N={N} nvfp4 2:4-pairs fused-rmsnorm",
                    "parallelism": f"replicas x{world}" if world > 1 else "single",
-                   "l2": f"{nsets} rotating input sets ({nsets * footprint / 2**20:.0f} MiB > L2)"},
+                   "l2": f"{nsets} rotating input sets ({nsets * footprint / 2**20:.0f} MiB > L2)",
+                   "launch": "device-timed legs replay one CUDA graph per step; e2e calls the API eagerly"},
         "eff_fp4_tflops": eff_tflops, "prep_gbs": prep_gbs,
         "t_prep_us": t_prep_ms * 1e3, "t_linear_us": t_lin_ms * 1e3,
         "roofline": dominant, "roofline_prep": rf_prep, "roofline_gemm": rf_gemm,

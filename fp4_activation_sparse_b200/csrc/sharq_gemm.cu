@@ -23,9 +23,11 @@
 //               Both paths carry the same per-row scale s_x, so one accumulator holds their
 //               sum. Each weight chunk feeds both MMAs. Commits arrive on both CTAs'
 //               barriers (multicast commit).
-//   warp 10     scale copier (leader): tcgen05.cp of the K step's scales and metadata into
-//               one of two tensor-memory buffers, from its own thread so that the copies of
-//               step k+1 are issued while the MMAs of step k run.
+//   warps 10-12 scale copiers (leader): tcgen05.cp of the K step's scales and metadata into one
+//               of three tensor-memory buffers -- dense-view weight scales (warp 10),
+//               sparse-view weight and backbone scales (warp 11), residual scales and metadata
+//               (warp 12) -- from their own threads: a copy costs its issuing thread tens of
+//               cycles, so three threads keep pace with the MMAs of the previous steps.
 //   warps 2..9  epilogue (both CTAs): tcgen05.ld of the whole accumulator into registers, release
 //               of the tensor memory, then y = acc * s_x[row] * s_w as bf16/fp32 stores while the
 //               next tile's MMAs run.
@@ -50,10 +52,13 @@ constexpr int BN = 256;   // output columns per pair tile
 constexpr int BK = 256;   // logical K per stage
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps + 32;  // producer, MMA, epilogue, scale copier
+constexpr int kCopiers = 3;
+constexpr int kThreads = 64 + 32 * kEpiWarps + 32 * kCopiers;  // producer, MMA, epilogue, scale copiers
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = 256;
-constexpr uint32_t kScaleBufCols = 80;  // per K-tile parity: meta 4, SFA_sp 8, SFA_res 16, SFB_sp 16, SFB_res 32
+constexpr uint32_t kScaleBufCols = 80;  // per buffer: meta 4, SFA_sp 8, SFA_res 16, SFB_sp 16, SFB_res 32
+constexpr uint32_t kScaleBufs = 3;      // 256 + 3 * 80 = 496 of 512 columns
+static_assert(kAccCols + kScaleBufs * kScaleBufCols <= kTmemCols, "tensor memory");
 // Drains (own copies and MMAs in flight before exit) always get the full bound, also when a
 // test lowers the limit of the ordinary waits.
 constexpr uint64_t kDrainLimitNs = 4000000000ull;
@@ -110,14 +115,25 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// CLUSTER: acquire at cluster scope, pairing with the peer CTA's release-arrive; otherwise
+// CTA scope (barriers completed by TMA transactions or tcgen05.commit).
+template <bool CLUSTER>
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
+  if (CLUSTER)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
   return ok != 0;
 }
 
@@ -129,12 +145,13 @@ __device__ __forceinline__ uint64_t globaltimer() {
 
 // Bounded wait: gives up after `limit_ns` (or when another role of the CTA already
 // gave up) and records the failure in the device status word.
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
                                           volatile uint32_t *abort_flag) {
-  if (mbar_try(bar, parity)) return true;
+  if (mbar_try<CLUSTER>(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try(bar, parity)) return true;
+    if (mbar_try<CLUSTER>(bar, parity)) return true;
     if (i == 1 || (i & 63u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > limit_ns) {
@@ -286,8 +303,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kMaxStageBytes);
-  // bars: full[kStages], empty[kStages], acc_full, acc_empty, drain, sf_full[kStages], sf_free[2], sf_drain
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 6);
+  // bars: full[kStages], empty[kStages], acc_full, acc_empty, drain, sf_full[kStages], sf_free[kScaleBufs],
+  // sf_drain[kCopiers]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 3 + kScaleBufs + kCopiers);
   volatile uint32_t *abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -299,8 +317,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
   const uint32_t acc_full = bar0 + 8u * (2 * kStages), acc_empty = acc_full + 8, drain_bar = acc_full + 16;
   auto sf_full_bar = [&](int s) { return bar0 + 8u * (2 * kStages + 3 + s); };
-  auto sf_free_bar = [&](int b) { return bar0 + 8u * (3 * kStages + 3 + b); };
-  const uint32_t sf_drain_bar = bar0 + 8u * (3 * kStages + 5);
+  auto sf_free_bar = [&](uint32_t b) { return bar0 + 8u * (3 * kStages + 3 + b); };
+  auto sf_drain_bar = [&](int c) { return bar0 + 8u * (3 * kStages + 3 + kScaleBufs + c); };
 
   using L = Stage<MX, SPARSE>;
   constexpr int apt_res = atoms_res(MX ? 1 : 0), apt_sp = atoms_sp(MX ? 1 : 0);
@@ -318,10 +336,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kEpiWarps);
     mbar_init(drain_bar, 1);
-    for (int s = 0; s < kStages; ++s) mbar_init(sf_full_bar(s), 1);
-    mbar_init(sf_free_bar(0), 1);
-    mbar_init(sf_free_bar(1), 1);
-    mbar_init(sf_drain_bar, 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(sf_full_bar(s), kCopiers);  // one commit per copier
+    for (uint32_t b = 0; b < kScaleBufs; ++b) mbar_init(sf_free_bar(b), 1);
+    for (int c = 0; c < kCopiers; ++c) mbar_init(sf_drain_bar(c), 1);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -385,20 +402,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer (leader CTA)
     if (lane == 0 && leader) {
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0, step = 0;
+      uint32_t phase = 0, acc_phase = 0, buf = 0;
       bool ok = true;
       const uint32_t acc = tmem;  // lanes 0..127 of each CTA, columns 0..255
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        if (!mbar_wait(acc_empty, acc_phase ^ 1u, limit, abort_flag)) { ok = false; break; }
+        // released by both CTAs' epilogue warps (remote arrives): cluster-scope acquire
+        if (!mbar_wait<true>(acc_empty, acc_phase ^ 1u, limit, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        for (int kt = 0; kt < num_k; ++kt, ++step) {
-          // the scale copier waited for this stage's bytes before copying its scales
+        for (int kt = 0; kt < num_k; ++kt) {
+          // the scale copiers waited for this stage's bytes before copying its scales
           if (!mbar_wait(sf_full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
           if (!mbar_wait(full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
           tc_fence_after();
           // descriptors: constant templates plus the operand's shared-memory address >> 4
           const uint32_t st4 = (smem0 + stage * kStageBytes) >> 4;
-          const uint32_t sbuf = tmem + kAccCols + (step & 1u) * kScaleBufCols;
+          const uint32_t sbuf = tmem + kAccCols + buf * kScaleBufCols;
           const uint32_t t_meta = sbuf, t_sfa_sp = sbuf + 4, t_sfa_res = sbuf + 12, t_sfb_sp = sbuf + 28,
                          t_sfb_res = sbuf + 44;
           constexpr int kA = 0, kW = L::kW;
@@ -427,7 +445,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             accumulate = 1u;
           }
           tc_commit_both(empty_bar(stage));  // frees the stage in both CTAs once these MMAs have read it
-          tc_commit_leader(sf_free_bar(step & 1u));  // and the scale buffer
+          tc_commit_leader(sf_free_bar(buf));  // and the scale buffer
+          if (++buf == kScaleBufs) buf = 0;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -453,100 +472,127 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float scale = row < p.T ? __fmul_rn(p.row_scale[row], s_w) : 0.f;
       if (!mbar_wait(acc_full, acc_phase, limit, abort_flag)) break;
       tc_fence_after();
-      // Read this warp's 32 rows x 128 columns of the accumulator, then hand the tensor memory
-      // back at once: the stores below overlap the next tile's MMAs.
-      uint32_t r[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32_async(tmem + ((uint32_t)(quarter * 32) << 16) + col_half * 128 + 32 * c, r[c]);
-      tmem_ld_wait();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence32(r[c]);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-      acc_phase ^= 1u;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int col = n0 + col_half * 128 + 32 * c;
-        if (row >= p.T || col >= p.N) continue;
-        if (p.out_f32) {
+      const uint32_t tacc = tmem + ((uint32_t)(quarter * 32) << 16) + col_half * 128;
+      const int col0 = n0 + col_half * 128;
+      const bool row_ok = row < p.T;
+      if (p.out_f32) {
+        // float32 output: 32 columns at a time, the tensor memory held until the last load
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32_async(tacc + 32 * c, r);
+          tmem_ld_wait();
+          reg_fence32(r);
+          const int col = col0 + 32 * c;
+          if (!row_ok || col >= p.N) continue;
           float *dst = reinterpret_cast<float *>(p.y) + (size_t)row * p.N + col;
           if (col + 32 <= p.N) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4 *>(dst + i) = make_float4(
-                  __fmul_rn(__uint_as_float(r[c][i]), scale), __fmul_rn(__uint_as_float(r[c][i + 1]), scale),
-                  __fmul_rn(__uint_as_float(r[c][i + 2]), scale), __fmul_rn(__uint_as_float(r[c][i + 3]), scale));
+              *reinterpret_cast<float4 *>(dst + i) =
+                  make_float4(__fmul_rn(__uint_as_float(r[i]), scale), __fmul_rn(__uint_as_float(r[i + 1]), scale),
+                              __fmul_rn(__uint_as_float(r[i + 2]), scale), __fmul_rn(__uint_as_float(r[i + 3]), scale));
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              if (col + i < p.N) dst[i] = __fmul_rn(__uint_as_float(r[c][i]), scale);
+              if (col + i < p.N) dst[i] = __fmul_rn(__uint_as_float(r[i]), scale);
           }
-        } else {
-          uint32_t packed[16];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+      } else {
+        // bf16 output: this warp's 32 rows x 128 columns are read and rounded first (64
+        // registers of packed pairs), the tensor memory is handed back, and the stores
+        // overlap the next tile's MMAs
+        uint32_t packed[4][16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32_async(tacc + 32 * c, r);
+          tmem_ld_wait();
+          reg_fence32(r);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[c][2 * i]), scale),
-                                                           __fmul_rn(__uint_as_float(r[c][2 * i + 1]), scale));
-            packed[i] = *reinterpret_cast<const uint32_t *>(&h);
+            const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * i]), scale),
+                                                           __fmul_rn(__uint_as_float(r[2 * i + 1]), scale));
+            packed[c][i] = *reinterpret_cast<const uint32_t *>(&h);
           }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int col = col0 + 32 * c;
+          if (!row_ok || col >= p.N) continue;
           uint16_t *dst = reinterpret_cast<uint16_t *>(p.y) + (size_t)row * p.N + col;
           if (col + 32 <= p.N) {
 #pragma unroll
             for (int i = 0; i < 16; i += 4)
-              *reinterpret_cast<uint4 *>(dst + 2 * i) = make_uint4(packed[i], packed[i + 1], packed[i + 2], packed[i + 3]);
+              *reinterpret_cast<uint4 *>(dst + 2 * i) =
+                  make_uint4(packed[c][i], packed[c][i + 1], packed[c][i + 2], packed[c][i + 3]);
           } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              if (col + 2 * i < p.N) *reinterpret_cast<uint32_t *>(dst + 2 * i) = packed[i];
+              if (col + 2 * i < p.N) *reinterpret_cast<uint32_t *>(dst + 2 * i) = packed[c][i];
           }
         }
       }
+      acc_phase ^= 1u;
     }
   }
 
   else {
-    // ------------------------------------------------------------ scale copier (warp 10, leader)
+    // ------------------------------------------------------------ scale copiers (warps 10..12; leader)
+    const int which = warp - (2 + kEpiWarps);
     if (lane == 0 && leader) {
       int stage = 0;
-      uint32_t phase = 0, step = 0;
+      uint32_t phase = 0, buf = 0, buf_phase = 0;
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        for (int kt = 0; kt < num_k; ++kt, ++step) {
+        for (int kt = 0; kt < num_k; ++kt) {
           if (!mbar_wait(full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
-          // buffer step%2 is free once the MMAs of step-2 completed
-          if (!mbar_wait(sf_free_bar(step & 1u), ((step >> 1) & 1u) ^ 1u, limit, abort_flag)) { ok = false; break; }
+          // the buffer is free once the MMAs that last read it (kScaleBufs steps ago) completed
+          if (!mbar_wait(sf_free_bar(buf), buf_phase ^ 1u, limit, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t st4 = (smem0 + stage * kStageBytes) >> 4;
-          const uint32_t sbuf = tmem + kAccCols + (step & 1u) * kScaleBufCols;
+          const uint32_t sbuf = tmem + kAccCols + buf * kScaleBufCols;
           const uint32_t t_meta = sbuf, t_sfa_sp = sbuf + 4, t_sfa_res = sbuf + 12, t_sfb_sp = sbuf + 28,
                          t_sfb_res = sbuf + 44;
           constexpr int kA = 0, kW = L::kW;
           // shared memory -> tensor memory (both CTAs). The weight chunk holds the scales of
           // both 128-row halves of the pair's 256 columns.
+          if (which == 0) {  // dense-view weight scales
 #pragma unroll
-          for (int a = 0; a < apt_res; ++a) {
-            tc_cp_atom(t_sfa_res + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_res + a * 512) / 16));
-            tc_cp_atom(t_sfb_res + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_res + a * 512) / 16));
-            tc_cp_atom(t_sfb_res + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_res + (apt_res + a) * 512) / 16));
-          }
-          if (SPARSE) {
-            tc_cp_128x128(t_meta, dsc(kDescNone, st4 + (kA + L::A.meta) / 16));
-#pragma unroll
-            for (int a = 0; a < apt_sp; ++a) {
-              tc_cp_atom(t_sfa_sp + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_sp + a * 512) / 16));
-              tc_cp_atom(t_sfb_sp + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_sp + a * 512) / 16));
-              tc_cp_atom(t_sfb_sp + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_sp + (apt_sp + a) * 512) / 16));
+            for (int a = 0; a < apt_res; ++a) {
+              tc_cp_atom(t_sfb_res + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_res + a * 512) / 16));
+              tc_cp_atom(t_sfb_res + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_res + (apt_res + a) * 512) / 16));
             }
+          } else if (which == 1) {  // sparse-view weight scales and backbone scales
+            if (SPARSE) {
+#pragma unroll
+              for (int a = 0; a < apt_sp; ++a) {
+                tc_cp_atom(t_sfb_sp + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_sp + a * 512) / 16));
+                tc_cp_atom(t_sfb_sp + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_sp + (apt_sp + a) * 512) / 16));
+                tc_cp_atom(t_sfa_sp + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_sp + a * 512) / 16));
+              }
+            }
+          } else {  // residual scales and metadata
+#pragma unroll
+            for (int a = 0; a < apt_res; ++a)
+              tc_cp_atom(t_sfa_res + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_res + a * 512) / 16));
+            if (SPARSE) tc_cp_128x128(t_meta, dsc(kDescNone, st4 + (kA + L::A.meta) / 16));
           }
           tc_commit_leader(sf_full_bar(stage));
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          if (++buf == kScaleBufs) { buf = 0; buf_phase ^= 1u; }
         }
       }
       // Drain: the copies issued above complete before TMEM is released.
-      tc_commit_leader(sf_drain_bar);
+      tc_commit_leader(sf_drain_bar(which));
       volatile uint32_t no_abort = 0;
-      mbar_wait(sf_drain_bar, 0, kDrainLimitNs, &no_abort);
+      mbar_wait(sf_drain_bar(which), 0, kDrainLimitNs, &no_abort);
     }
   }
 
@@ -586,20 +632,61 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Host-side launch cost matters at these kernel durations (tens of microseconds): tensor
+// maps are cached by (base, rows, box) -- a map encodes nothing but the address and shape --
+// and the per-device setup (shared-memory opt-in, SM count) is done once per device.
+struct MapCache {
+  struct Entry {
+    const void *base;
+    uint64_t rows;
+    uint32_t box_rows;
+    CUtensorMap map;
+  };
+  static constexpr int kEntries = 32;
+  std::mutex mu;
+  Entry e[kEntries];
+  int used = 0, next = 0;
+
+  bool get(CUtensorMap *out, const void *base, uint64_t rows, uint32_t box_rows) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+      if (e[i].base == base && e[i].rows == rows && e[i].box_rows == box_rows) {
+        *out = e[i].map;
+        return true;
+      }
+    // chunk rows of 1024 bytes (256 x u32), one box = one chunk
+    if (!make_map(out, base, CU_TENSOR_MAP_DATA_TYPE_UINT32, 256, rows, 256, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+    Entry &slot = e[used < kEntries ? used++ : next];
+    if (used == kEntries) next = (next + 1) % kEntries;
+    slot.base = base;
+    slot.rows = rows;
+    slot.box_rows = box_rows;
+    slot.map = *out;
+    return true;
+  }
+};
+
+constexpr int kMaxDevices = 64;
+
 template <bool MX, bool SPARSE>
 cudaError_t launch_t(const TmaMaps &maps, const GemmParams &p, cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(sharq_gemm_kernel<MX, SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t setup_err[kMaxDevices];
+  static int sms[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [dev] {
+    setup_err[dev] = cudaFuncSetAttribute(sharq_gemm_kernel<MX, SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          kSmemBytes);
+    if (setup_err[dev] == cudaSuccess)
+      setup_err[dev] = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+  });
+  if (setup_err[dev] != cudaSuccess) return setup_err[dev];
   const int tiles = ((p.T + 2 * BM - 1) / (2 * BM)) * ((p.N + BN - 1) / BN);
-  const int pairs = tiles < sms / 2 ? tiles : sms / 2;
+  const int pairs = tiles < sms[dev] / 2 ? tiles : sms[dev] / 2;
   sharq_gemm_kernel<MX, SPARSE><<<2 * pairs, kThreads, kSmemBytes, st>>>(maps, p);
   return cudaGetLastError();
 }
@@ -607,18 +694,15 @@ cudaError_t launch_t(const TmaMaps &maps, const GemmParams &p, cudaStream_t st) 
 }  // namespace
 
 cudaError_t launch_gemm(const GemmParams &p, cudaStream_t st, const char **why) {
+  static MapCache cache;
   TmaMaps maps;
-  memset(&maps, 0, sizeof maps);
   const int fmt = p.fmt == kFmtMX ? 1 : 0;
   const ActTile A = act_tile(fmt, 2, p.sparse != 0);
   const WTile W = w_tile(fmt);
   const uint64_t ks = (uint64_t)p.K / BK;
   const uint64_t a_rows = (uint64_t)(p.T_pad / 128) * ks * (A.bytes / 1024);
   const uint64_t w_rows = (uint64_t)(p.N_pad / 128) * ks * (W.bytes / 1024);
-  const auto U32 = CU_TENSOR_MAP_DATA_TYPE_UINT32;
-  const bool ok = make_map(&maps.act, p.a_tiles, U32, 256, a_rows, 256, A.bytes / 1024, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-                  make_map(&maps.w, p.w_tiles, U32, 256, w_rows, 256, W.bytes / 1024, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (!ok) {
+  if (!cache.get(&maps.act, p.a_tiles, a_rows, A.bytes / 1024) || !cache.get(&maps.w, p.w_tiles, w_rows, W.bytes / 1024)) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or operand layout rejected)";
     return cudaErrorInvalidValue;
   }

@@ -21,6 +21,8 @@
 // and 128x4 scale atoms: the GEMM's shared-memory image); rows T..T_pad-1 are zeroed. The RMSNorm weight is staged once
 // per block in shared memory as float32. Float32 arithmetic uses explicit
 // round-to-nearest scalar operations, so no contraction changes a rounding.
+#include <mutex>
+
 #include "sharq_common.cuh"
 #include "sharq_internal.h"
 
@@ -419,9 +421,18 @@ cudaError_t launch_t(const PrepParams &p, cudaStream_t st) {
   // the staging layout reserves 512 floats per 32 double pieces: round K up to 512
   const size_t smem = NORM ? (size_t)((p.K + 511) / 512 * 512) * sizeof(float) : 0;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(prep_kernel<FMT, UNIT, NORM, DENSE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // opt in once per device to the largest staging size (K = 32768)
+    static std::once_flag once[64];
+    static cudaError_t err[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [dev] {
+      err[dev] = cudaFuncSetAttribute(prep_kernel<FMT, UNIT, NORM, DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      32768 * (int)sizeof(float));
+    });
+    if (err[dev] != cudaSuccess) return err[dev];
   }
   prep_kernel<FMT, UNIT, NORM, DENSE><<<grid, block, smem, st>>>(p);
   return cudaGetLastError();
