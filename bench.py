@@ -16,8 +16,10 @@ independent, every rank processes its own batch with no data-path collective
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -102,21 +104,52 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
-def dist_setup(n_gpus: int):
+CSRC = os.path.join(ROOT, "fp4_activation_sparse_b200", "csrc")
+
+
+def profiled_traffic(profile: str, sources: list[str], rows: int) -> float | None:
+    """DRAM bytes (read + write) per launch from a committed ncu summary under profiles/, or
+    None when the kernel's sources changed since the capture (hash recorded in the summary)."""
+    try:
+        text = open(os.path.join(ROOT, "profiles", profile)).read()
+    except OSError:
+        return None
+    m = re.search(r"sha256\[:16\][^:]*: ([0-9a-f]{16})", text)
+    h = hashlib.sha256()
+    for f in sources:
+        h.update(open(os.path.join(CSRC, f), "rb").read())
+    if not m or m.group(1) != h.hexdigest()[:16]:
+        return None
+    if (t := re.search(r"traffic_bytes_per_launch: (\d+)", text)):
+        return float(t.group(1))
+    if (t := re.search(r"traffic_bytes_per_row: (\d+)", text)):
+        return float(t.group(1)) * rows
+    return None
+
+
+def dist_setup(n_gpus: int, backend: str | None = None):
+    """One process per GPU (torchrun env). Replicas: no data-path collective; the process
+    group carries only the barrier and the max-over-ranks of the timings."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        backend = backend or "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return rank, world, local
+
+
+def _reduce_device() -> str:
+    return "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
 
 
 def max_over_ranks(v: float, world: int) -> float:
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_reduce_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -124,6 +157,16 @@ def max_over_ranks(v: float, world: int) -> float:
 def barrier(world: int):
     if world > 1:
         torch.distributed.barrier()
+
+
+def replica_seed(rank: int) -> int:
+    """Each replica draws its own synthetic batch (weak scaling: fixed work per GPU)."""
+    return 1 + rank
+
+
+def aggregate_tokens_per_s(tokens_per_step: int, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's device time."""
+    return tokens_per_step * steps * world / (ms_max / 1e3)
 
 
 def to_dev(bits: np.ndarray) -> torch.Tensor:
@@ -188,7 +231,7 @@ def run_sharq(args, rank, world, local):
     hbm_peak, bf16_peak, bf16_sust, peak_src = load_peaks()
     fp4_dense_peak = bf16_peak * 4.0  # nominal FP4:BF16 dense ratio 9 : 2.25 applied to the measured bf16 peak
 
-    lin = wl.llama_qkv(T=2048, seed=1 + rank)
+    lin = wl.llama_qkv(T=2048, seed=replica_seed(rank))
     T, K, N = lin.shape
     # input sets rotated so each step touches data last used > L2 bytes earlier
     w_dev = to_dev(lin.w)
@@ -329,17 +372,20 @@ def run_sharq(args, rank, world, local):
     if rank != 0:
         return
     tokens = T * args.steps * world
-    value = tokens / (ms_total / 1e3)
+    value = aggregate_tokens_per_s(T, args.steps, world, ms_total)
     eff_tflops = 2.0 * T * N * K * args.steps * world / (ms_total / 1e3) / 1e12
     prep_bytes = T * K * PREP_BYTES_PER_ELEM + T * 4 + K * 2
     prep_gbs = prep_bytes / (t_prep_ms / 1e3) / 1e9
     gemm_work = 3.0 * T * N * K  # dense-equivalent tensor work: sparse path T*N*K, dense path 2*T*N*K
     gemm_tflops = gemm_work / (t_lin_ms / 1e3) / 1e12
+    common = ["sharq_common.cuh", "sharq_internal.h"]
     rf_prep = {"bound": "hbm", "achieved": prep_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": prep_gbs / hbm_peak,
-               "traffic": None, "kernel": "sharq_prep", "peak_source": peak_src}
+               "traffic": profiled_traffic("prep_kernel_llama_qkv_T16384.md", ["sharq_prep.cu"] + common, T),
+               "kernel": "sharq_prep", "peak_source": peak_src}
     rf_gemm = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_dense_peak, "unit": "TFLOP/s",
-               "frac": gemm_tflops / fp4_dense_peak, "traffic": None, "kernel": "sharq_gemm",
-               "peak_source": f"{peak_src} bf16 x 4 (nominal dense FP4:BF16)"}
+               "frac": gemm_tflops / fp4_dense_peak,
+               "traffic": profiled_traffic("sharq_gemm_llama_qkv_T2048.md", ["sharq_gemm.cu"] + common, T),
+               "kernel": "sharq_gemm", "peak_source": f"{peak_src} bf16 x 4 (nominal dense FP4:BF16)"}
     dominant = rf_gemm if t_lin_ms >= t_prep_ms else rf_prep
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -378,7 +424,7 @@ def run_profile(args):
     x, g, w = to_dev(lin.x), to_dev(lin.gamma), to_dev(lin.w)
     wp = S.sharq_pack_weight(w, "nvfp4")
     p = S.sharq_prepare(x, g, lin.eps)
-    q = S.sharq_quantize_dense(x, g, lin.eps)
+    q = S.sharq_quantize_dense(x, g, lin.eps) if args.profile == "dense" else None
     y = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
     for _ in range(3):
         if args.profile == "prep":
