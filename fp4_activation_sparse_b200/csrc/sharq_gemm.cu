@@ -23,11 +23,12 @@
 //               Both paths carry the same per-row scale s_x, so one accumulator holds their
 //               sum. Each weight chunk feeds both MMAs. Commits arrive on both CTAs'
 //               barriers (multicast commit).
-//   warps 10-12 scale copiers (leader): tcgen05.cp of the K step's scales and metadata into one
-//               of three tensor-memory buffers -- dense-view weight scales (warp 10),
-//               sparse-view weight and backbone scales (warp 11), residual scales and metadata
-//               (warp 12) -- from their own threads: a copy costs its issuing thread tens of
-//               cycles, so three threads keep pace with the MMAs of the previous steps.
+//   warps 10-14 scale copiers (leader): tcgen05.cp of the K step's scales and metadata into one
+//               of three tensor-memory buffers, split five ways (dense-view weight scales of
+//               the first and second K halves, sparse-view weight scales, residual scales,
+//               backbone scales + metadata), each from its own thread: a copy costs its
+//               issuing thread tens of cycles, so the copies keep pace with the MMAs only
+//               when spread over several threads.
 //   warps 2..9  epilogue (both CTAs): tcgen05.ld of the whole accumulator into registers, release
 //               of the tensor memory, then y = acc * s_x[row] * s_w as bf16/fp32 stores while the
 //               next tile's MMAs run.
@@ -52,7 +53,7 @@ constexpr int BN = 256;   // output columns per pair tile
 constexpr int BK = 256;   // logical K per stage
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;
-constexpr int kCopiers = 3;
+constexpr int kCopiers = 5;
 constexpr int kThreads = 64 + 32 * kEpiWarps + 32 * kCopiers;  // producer, MMA, epilogue, scale copiers
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = 256;
@@ -507,17 +508,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // overlap the next tile's MMAs
         uint32_t packed[4][16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32_async(tacc + 32 * c, r);
+        for (int h = 0; h < 2; ++h) {  // two loads in flight per wait
+          uint32_t r[2][32];
+          tmem_ld32_async(tacc + 64 * h, r[0]);
+          tmem_ld32_async(tacc + 64 * h + 32, r[1]);
           tmem_ld_wait();
-          reg_fence32(r);
+          reg_fence32(r[0]);
+          reg_fence32(r[1]);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * i]), scale),
-                                                           __fmul_rn(__uint_as_float(r[2 * i + 1]), scale));
-            packed[c][i] = *reinterpret_cast<const uint32_t *>(&h);
-          }
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const __nv_bfloat162 v = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[c][2 * i]), scale),
+                                                             __fmul_rn(__uint_as_float(r[c][2 * i + 1]), scale));
+              packed[2 * h + c][i] = *reinterpret_cast<const uint32_t *>(&v);
+            }
         }
         tc_fence_before();
         __syncwarp();
@@ -544,7 +549,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 
   else {
-    // ------------------------------------------------------------ scale copiers (warps 10..12; leader)
+    // ------------------------------------------------------------ scale copiers (warps 10..14; leader)
     const int which = warp - (2 + kEpiWarps);
     if (lane == 0 && leader) {
       int stage = 0;
@@ -563,26 +568,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           constexpr int kA = 0, kW = L::kW;
           // shared memory -> tensor memory (both CTAs). The weight chunk holds the scales of
           // both 128-row halves of the pair's 256 columns.
-          if (which == 0) {  // dense-view weight scales
+          if (which < 2) {  // dense-view weight scales, one K half each (both 128-row n-blocks)
 #pragma unroll
-            for (int a = 0; a < apt_res; ++a) {
+            for (int a = which * apt_res / 2; a < (which + 1) * apt_res / 2; ++a) {
               tc_cp_atom(t_sfb_res + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_res + a * 512) / 16));
               tc_cp_atom(t_sfb_res + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_res + (apt_res + a) * 512) / 16));
             }
-          } else if (which == 1) {  // sparse-view weight scales and backbone scales
+          } else if (which == 2) {  // sparse-view weight scales
             if (SPARSE) {
 #pragma unroll
               for (int a = 0; a < apt_sp; ++a) {
                 tc_cp_atom(t_sfb_sp + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_sp + a * 512) / 16));
                 tc_cp_atom(t_sfb_sp + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_sp + (apt_sp + a) * 512) / 16));
-                tc_cp_atom(t_sfa_sp + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_sp + a * 512) / 16));
               }
             }
-          } else {  // residual scales and metadata
+          } else if (which == 3) {  // residual scales
 #pragma unroll
             for (int a = 0; a < apt_res; ++a)
               tc_cp_atom(t_sfa_res + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_res + a * 512) / 16));
-            if (SPARSE) tc_cp_128x128(t_meta, dsc(kDescNone, st4 + (kA + L::A.meta) / 16));
+          } else if (SPARSE) {  // backbone scales and metadata
+#pragma unroll
+            for (int a = 0; a < apt_sp; ++a)
+              tc_cp_atom(t_sfa_sp + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_sp + a * 512) / 16));
+            tc_cp_128x128(t_meta, dsc(kDescNone, st4 + (kA + L::A.meta) / 16));
           }
           tc_commit_leader(sf_full_bar(stage));
           if (++stage == kStages) { stage = 0; phase ^= 1u; }

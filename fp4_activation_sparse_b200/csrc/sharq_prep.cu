@@ -20,7 +20,12 @@
 // tiled activation operand (chunks of 128 rows x 256 K holding swizzled codes, metadata
 // and 128x4 scale atoms: the GEMM's shared-memory image); rows T..T_pad-1 are zeroed. The RMSNorm weight is staged once
 // per block in shared memory as float32. Float32 arithmetic uses explicit
-// round-to-nearest scalar operations, so no contraction changes a rounding.
+// round-to-nearest operations so that no contraction changes a rounding: scalar mul.rn /
+// sub.rn, or the packed f32x2 forms, which round each lane exactly like the scalar ones
+// (checked bitwise on B200 over random finite operands, subnormals, signed zeros and
+// infinities) but which the assembler may fuse into a packed FMA when a packed product
+// feeds a packed add. So a packed product never feeds an addition here: products that do
+// (x*rstd*gamma and the dequantized backbone, both subtracted for the residual) are scalar.
 #include <mutex>
 
 #include "sharq_common.cuh"
@@ -55,6 +60,29 @@ __device__ __forceinline__ void ld256(const void *p, uint32_t (&r)[8]) {
                : "l"(p));
 }
 
+// Packed float32 pairs: (a, b) op= (c, d), each lane rounded to nearest even.
+__device__ __forceinline__ void mul2(float &a, float &b, float c, float d) {
+  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\tmul.rn.f32x2 z, x, y;\n\t"
+      "mov.b64 {%0, %1}, z;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(c), "f"(d));
+}
+__device__ __forceinline__ void sub2(float &a, float &b, float c, float d) {
+  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\tsub.rn.f32x2 z, x, y;\n\t"
+      "mov.b64 {%0, %1}, z;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(c), "f"(d));
+}
+
+// Exact squares of a word's two bf16 values added to a float64 sum (low half first).
+__device__ __forceinline__ double add_squares(uint32_t w, double ss) {
+  double lo, hi;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f64.bf16 %0, l;\n\tcvt.f64.bf16 %1, h;\n\t}"
+      : "=d"(lo), "=d"(hi)
+      : "r"(w));
+  return __fma_rn(hi, hi, __fma_rn(lo, lo, ss));
+}
+
 __device__ __forceinline__ void unpack16(const uint32_t (&w)[8], float *v) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -71,16 +99,25 @@ __device__ __forceinline__ int gamma_smem_index(int k) {
   return ((((dp >> 5) << 2) + c) * 32 + (dp & 31)) * 4 + (k & 3);
 }
 
-// xh = fp32(fp32(x * rstd) * gamma) for the 16 values of double piece dp
-__device__ __forceinline__ void normalize16(float *v, const float *gs, int dp, float rstd) {
-  const float4 *g4 = reinterpret_cast<const float4 *>(gs);
+// xh = fp32(fp32(x * rstd) * gamma) for the 16 values of a double piece whose staged weights
+// start at g4 (this lane's chunk 0; chunk c at g4 + 32 c). PACKED_GAMMA: the gamma product
+// may be packed (its result feeds no addition: the row-amax pass).
+template <bool PACKED_GAMMA>
+__device__ __forceinline__ void normalize16(float *v, const float4 *g4, float rstd) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    const float4 g = g4[(((dp >> 5) << 2) + c) * 32 + (dp & 31)];
-    v[4 * c + 0] = __fmul_rn(__fmul_rn(v[4 * c + 0], rstd), g.x);
-    v[4 * c + 1] = __fmul_rn(__fmul_rn(v[4 * c + 1], rstd), g.y);
-    v[4 * c + 2] = __fmul_rn(__fmul_rn(v[4 * c + 2], rstd), g.z);
-    v[4 * c + 3] = __fmul_rn(__fmul_rn(v[4 * c + 3], rstd), g.w);
+    const float4 g = g4[32 * c];
+    mul2(v[4 * c + 0], v[4 * c + 1], rstd, rstd);
+    mul2(v[4 * c + 2], v[4 * c + 3], rstd, rstd);
+    if (PACKED_GAMMA) {
+      mul2(v[4 * c + 0], v[4 * c + 1], g.x, g.y);
+      mul2(v[4 * c + 2], v[4 * c + 3], g.z, g.w);
+    } else {
+      v[4 * c + 0] = __fmul_rn(v[4 * c + 0], g.x);
+      v[4 * c + 1] = __fmul_rn(v[4 * c + 1], g.y);
+      v[4 * c + 2] = __fmul_rn(v[4 * c + 2], g.z);
+      v[4 * c + 3] = __fmul_rn(v[4 * c + 3], g.w);
+    }
   }
 }
 
@@ -122,7 +159,11 @@ __device__ __forceinline__ MxScale mx_scale(float amax) {
 __device__ __forceinline__ void codes16(const float *v, float mult, uint32_t &w0, uint32_t &w1) {
   float t[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) t[i] = __fmul_rn(v[i], mult);
+  for (int i = 0; i < 16; i += 2) {
+    t[i] = v[i];
+    t[i + 1] = v[i + 1];
+    mul2(t[i], t[i + 1], mult, mult);
+  }
   w0 = cvt_e2m1x8(t[0], t[1], t[2], t[3], t[4], t[5], t[6], t[7]);
   w1 = cvt_e2m1x8(t[8], t[9], t[10], t[11], t[12], t[13], t[14], t[15]);
 }
@@ -138,7 +179,7 @@ __device__ __forceinline__ void deq8(uint32_t w, float dec, float s_x, float *o)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const __half2 q = __hmul2(*reinterpret_cast<const __half2 *>(&h[j]), d2);  // exact (<= 6 significant bits)
-      const float2 f = __half22float2(q);
+      const float2 f = __half22float2(q);  // scalar products: they feed the residual subtraction
       o[2 * j] = __fmul_rn(f.x, s_x);
       o[2 * j + 1] = __fmul_rn(f.y, s_x);
     }
@@ -152,52 +193,53 @@ __device__ __forceinline__ void deq8(uint32_t w, float dec, float s_x, float *o)
   }
 }
 
-// Where double piece dp (16 K positions) of a row lands in the tiled operand: its chunk
-// (128-row block, 256-K step), the row inside the block and the piece inside the step.
+// Where a lane's double pieces land in the tiled operand. A lane's pieces dp = i*32W + 32wt +
+// lane all have the same position j = dp % 16 inside their 256-K step (32W and 32 are
+// multiples of 16) and the same row, so every offset inside a chunk is fixed per lane; only
+// the chunk changes from piece to piece.
 struct Spot {
-  uint8_t *chunk;
-  int r, j;
+  int res, sp, meta, sf_sp, sf_res;  // byte offsets inside a chunk (sf_*: -1 = no scale byte here)
 };
 template <int FMT, int UNIT, bool DENSE>
-__device__ __forceinline__ Spot spot(const PrepParams &p, int row, int dp) {
+__device__ __forceinline__ Spot lane_spot(int row, int lane) {
   constexpr ActTile L = act_tile(FMT, UNIT, !DENSE);
-  Spot s;
-  s.chunk = p.tiles + ((size_t)(row >> 7) * p.KS + (dp >> 4)) * L.bytes;
-  s.r = row & 127;
-  s.j = dp & 15;
-  return s;
+  const int r = row & 127, j = lane & 15;
+  Spot o;
+  // 128-byte rows, 16-byte unit j/2 swizzled with row bits 0..2
+  o.res = L.res + r * 128 + (((j >> 1) ^ (r & 7)) << 4) + (j & 1) * 8;
+  // 64-byte rows, 16-byte unit j/4 swizzled with row bits 1..2
+  o.sp = L.sp + r * 64 + (((j >> 2) ^ ((r >> 1) & 3)) << 4) + (j & 3) * 4;
+  o.meta = UNIT == 2 ? L.meta + r * 16 + j : L.meta + (j >> 3) * 2048 + r * 16 + (j & 7) * 2;
+  if (FMT == kFmtNV) {  // one backbone scale per 2 pieces, one residual scale per piece
+    o.sf_sp = (j & 1) == 0 ? L.sf_sp + atom_pos(r, j >> 1) : -1;
+    o.sf_res = L.sf_res + atom_pos(r, j);
+  } else {  // one backbone scale per 4 pieces, one residual scale per 2
+    o.sf_sp = (j & 3) == 0 ? L.sf_sp + atom_pos(r, j >> 2) : -1;
+    o.sf_res = (j & 1) == 0 ? L.sf_res + atom_pos(r, j >> 1) : -1;
+  }
+  return o;
 }
 
-// Store the results of one double piece: backbone codes (4 bytes: 8 kept values), its
-// metadata (pair unit 8 bits, element unit 16 bits), the backbone block scale (written by
-// the first lane of its block), residual codes (8 bytes) and residual block scale.
+// Store the results of one double piece into its chunk: backbone codes (4 bytes: 8 kept
+// values), metadata (pair unit 8 bits, element unit 16 bits), the backbone block scale (first
+// lane of its block), residual codes (8 bytes) and the residual block scale.
 template <int FMT, int UNIT, bool DENSE>
-__device__ __forceinline__ void store16(const Spot &o, uint32_t kept, uint32_t meta, uint32_t sc_sp, uint32_t r0,
-                                        uint32_t r1, uint32_t sc_res) {
-  constexpr ActTile L = act_tile(FMT, UNIT, !DENSE);
-  const int r = o.r, j = o.j;
+__device__ __forceinline__ void store16(uint8_t *chunk, const Spot &o, uint32_t kept, uint32_t meta, uint32_t sc_sp,
+                                        uint32_t r0, uint32_t r1, uint32_t sc_res) {
   if (!DENSE) {
-    // 64-byte rows, 16-byte unit j/4 swizzled with row bits 1..2
-    *reinterpret_cast<uint32_t *>(o.chunk + L.sp + r * 64 + (((j >> 2) ^ ((r >> 1) & 3)) << 4) + (j & 3) * 4) = kept;
-    if (UNIT == 2) o.chunk[L.meta + r * 16 + j] = (uint8_t)meta;
-    else *reinterpret_cast<uint16_t *>(o.chunk + L.meta + (j >> 3) * 2048 + r * 16 + (j & 7) * 2) = (uint16_t)meta;
-    if (FMT == kFmtNV) {  // one backbone scale per 2 pieces
-      if ((j & 1) == 0) o.chunk[L.sf_sp + atom_pos(r, j >> 1)] = (uint8_t)sc_sp;
-    } else if ((j & 3) == 0) {  // one per 4 pieces
-      o.chunk[L.sf_sp + atom_pos(r, j >> 2)] = (uint8_t)sc_sp;
-    }
+    *reinterpret_cast<uint32_t *>(chunk + o.sp) = kept;
+    if (UNIT == 2) chunk[o.meta] = (uint8_t)meta;
+    else *reinterpret_cast<uint16_t *>(chunk + o.meta) = (uint16_t)meta;
+    if (o.sf_sp >= 0) chunk[o.sf_sp] = (uint8_t)sc_sp;
   }
-  // 128-byte rows, 16-byte unit j/2 swizzled with row bits 0..2
-  *reinterpret_cast<uint2 *>(o.chunk + L.res + r * 128 + (((j >> 1) ^ (r & 7)) << 4) + (j & 1) * 8) =
-      make_uint2(r0, r1);
-  if (FMT == kFmtNV) o.chunk[L.sf_res + atom_pos(r, j)] = (uint8_t)sc_res;
-  else if ((j & 1) == 0) o.chunk[L.sf_res + atom_pos(r, j >> 1)] = (uint8_t)sc_res;
+  *reinterpret_cast<uint2 *>(chunk + o.res) = make_uint2(r0, r1);
+  if (o.sf_res >= 0) chunk[o.sf_res] = (uint8_t)sc_res;
 }
 
 // ---------------------------------------------------------------- one double piece
 // 16 normalized values of double piece `dp` (lane-aligned: dp % 32 == lane).
 template <int FMT, int UNIT, bool DENSE>
-__device__ __forceinline__ void process16(const PrepParams &p, float *v, int row, int dp, bool live, float s_x,
+__device__ __forceinline__ void process16(uint8_t *chunk, const Spot &o, float *v, bool live, float s_x,
                                           float g_x) {
   uint32_t kept = 0u, meta = 0u, sc_sp = 0u;
   if (!DENSE) {
@@ -267,7 +309,7 @@ __device__ __forceinline__ void process16(const PrepParams &p, float *v, int row
     deq8<FMT>(w0, dec, s_x, dq);
     deq8<FMT>(w1, dec, s_x, dq + 8);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __fsub_rn(v[i], dq[i]);
+    for (int i = 0; i < 16; i += 2) sub2(v[i], v[i + 1], dq[i], dq[i + 1]);
   }
   // ---- residual (or xh itself for the dense quantizer): dense blocks
   float am = 0.f;
@@ -286,7 +328,7 @@ __device__ __forceinline__ void process16(const PrepParams &p, float *v, int row
     if (s.zero) { r0 = 0u; r1 = 0u; }
     sc_res = s.code;
   }
-  if (live) store16<FMT, UNIT, DENSE>(spot<FMT, UNIT, DENSE>(p, row, dp), kept, meta, sc_sp, r0, r1, sc_res);
+  if (live) store16<FMT, UNIT, DENSE>(chunk, o, kept, meta, sc_sp, r0, r1, sc_res);
 }
 
 // ---------------------------------------------------------------- team reductions
@@ -329,7 +371,7 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   extern __shared__ float4 gamma_smem4[];  // NORM: the RMSNorm weight as float32 (K rounded up to 512)
   __shared__ double sm_d[64];
   __shared__ float sm_f[64];
-  float *gs = reinterpret_cast<float *>(gamma_smem4);
+  float *gs = reinterpret_cast<float *>(gamma_smem4);  // [dp/32][chunk][lane][4] (gamma_smem_index)
   const int W = p.TS;  // warps per row team
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int team = warp / W, wt = warp - team * W;
@@ -358,12 +400,10 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
     for (int i = 0; i < kMaxDP; ++i) {
       const int dp = i * stride + wt * 32 + lane;
       if (live_row && dp < ndp_row) {
-        float v[16];
-        unpack16(xr[i], v);
-        // float64 per element: bf16 squares are exact and the sum keeps ~2^-53 relative
-        // accuracy, so fp32(sum/K) does not depend on the summation order in practice
+        // float64: bf16 squares are exact and the sum keeps ~2^-53 relative accuracy, so
+        // fp32(sum/K) does not depend on the summation order in practice
 #pragma unroll
-        for (int j = 0; j < 16; ++j) ss = __fma_rn((double)v[j], (double)v[j], ss);
+        for (int w = 0; w < 8; ++w) ss = add_squares(xr[i][w], ss);
       }
     }
     __syncthreads();  // gamma staged
@@ -371,6 +411,8 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
     const float ms = __double2float_rn(__ddiv_rn(ss, (double)p.K));
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, p.eps)));
   }
+  // staged weights of this lane's piece i: chunk c at g_lane + i*128W + 32c (see gamma_smem_index)
+  const float4 *g_lane = gamma_smem4 + wt * 128 + lane;
 
   float am = 0.f;
 #pragma unroll
@@ -379,7 +421,7 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
     if (live_row && dp < ndp_row) {
       float v[16];
       unpack16(xr[i], v);
-      if (NORM) normalize16(v, gs, dp, rstd);
+      if (NORM) normalize16<true>(v, g_lane + i * 128 * W, rstd);
 #pragma unroll
       for (int j = 0; j < 16; ++j) am = fmaxf(am, fabsf(v[j]));
     }
@@ -388,6 +430,11 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   float s_x, g_x;
   row_scales(FMT, am, s_x, g_x);
 
+  constexpr int kChunk = act_tile(FMT, UNIT, !DENSE).bytes;
+  const Spot o = lane_spot<FMT, UNIT, DENSE>(row, lane);
+  // chunk of piece i: row block, then K step i*2W + 2wt + lane/16
+  uint8_t *chunk0 = p.tiles + ((size_t)(row >> 7) * p.KS + 2 * wt + (lane >> 4)) * kChunk;
+  const size_t chunk_step = (size_t)2 * W * kChunk;
   const bool pad_row = !live_row && row < p.T_pad;
 #pragma unroll
   for (int i = 0; i < kMaxDP; ++i) {
@@ -395,18 +442,19 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
     if (base >= ndp_row) break;
     const int dp = base + lane;
     const bool live = live_row && dp < ndp_row;
+    uint8_t *chunk = chunk0 + i * chunk_step;
     if (live_row) {
       float v[16];
       if (live) {
         unpack16(xr[i], v);
-        if (NORM) normalize16(v, gs, dp, rstd);
+        if (NORM) normalize16<false>(v, g_lane + i * 128 * W, rstd);
       } else {
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = 0.f;
       }
-      process16<FMT, UNIT, DENSE>(p, v, row, dp, live, s_x, g_x);
+      process16<FMT, UNIT, DENSE>(chunk, o, v, live, s_x, g_x);
     } else if (pad_row && dp < ndp_row) {
-      store16<FMT, UNIT, DENSE>(spot<FMT, UNIT, DENSE>(p, row, dp), 0u, 0u, 0u, 0u, 0u, 0u);
+      store16<FMT, UNIT, DENSE>(chunk, o, 0u, 0u, 0u, 0u, 0u, 0u);
     }
   }
   if (live_row && wt == 0 && lane == 0) p.row_scale[row] = s_x;
