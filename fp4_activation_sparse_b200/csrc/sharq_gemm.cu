@@ -29,9 +29,12 @@
 //               backbone scales + metadata), each from its own thread: a copy costs its
 //               issuing thread tens of cycles, so the copies keep pace with the MMAs only
 //               when spread over several threads.
-//   warps 2..9  epilogue (both CTAs): tcgen05.ld of the whole accumulator into registers, release
-//               of the tensor memory, then y = acc * s_x[row] * s_w as bf16/fp32 stores while the
-//               next tile's MMAs run.
+//   warps 2..9  epilogue (both CTAs): tcgen05.ld of the accumulator, y = acc * s_x[row] * s_w
+//               rounded to bf16 in registers, the tensor memory handed back, then the block
+//               staged in shared memory and written by bulk tensor stores (coalesced, clipped at
+//               the tensor's edges) while the next tile's MMAs run. Row-wise 16-byte stores
+//               from registers took a quarter of the kernel's time and delayed the next tile's
+//               loads. (float32 output, a test format, is stored from registers.)
 // Every mbarrier wait is bounded by a time limit; on expiry the CTA records a status word,
 // stops issuing, drains (bounded) what it issued, frees TMEM and exits.
 #include <cuda.h>
@@ -73,12 +76,18 @@ struct Stage {
   static constexpr int kBytes = A.bytes + W.bytes;
 };
 constexpr int kMaxStageBytes = 52224;  // NVFP4 SharQ: 29696 + 22528
-constexpr int kSmemBytes = kStages * kMaxStageBytes + 1024 /*align slack*/ + 256 /*barriers*/;
+// bf16 output staging for the epilogue's bulk tensor stores: per epilogue warp one box of 32
+// rows x 32 columns (64-byte rows, 64-byte swizzle), reused four times per tile
+constexpr int kStageOutBytes = 2048;
+constexpr int kOutOffset = kStages * kMaxStageBytes;  // 1024-aligned
+constexpr int kSmemBytes = kOutOffset + kEpiWarps * kStageOutBytes + 1024 /*align slack*/ + 256 /*barriers*/;
 static_assert(Stage<false, true>::kBytes <= kMaxStageBytes && Stage<true, true>::kBytes <= kMaxStageBytes, "stage");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kOutOffset % 1024 == 0, "staging alignment");
 
 struct __align__(64) TmaMaps {
   CUtensorMap act, w;  // both: rows of 1024 bytes (256 x u32), one box = one chunk
+  CUtensorMap y;       // bf16 output [T][N], box 32 columns x 32 rows, 64-byte swizzle
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -193,6 +202,19 @@ __device__ __forceinline__ void tc_commit_both(uint32_t bar) {
       : "memory");
 }
 
+// 2-D bulk tensor store from this CTA's shared memory (completion tracked by bulk groups)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(c0),
+               "r"(c1), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until the committed stores have finished reading shared memory / have completed
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// generic-proxy shared-memory writes become visible to the bulk-copy (async) proxy
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // arrive once on the leader CTA's barrier at this offset when this thread's tcgen05 operations finish
 __device__ __forceinline__ void tc_commit_leader(uint32_t bar) {
   const uint16_t mask = 0x1;
@@ -303,7 +325,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     sharq_gemm_kernel(const __grid_constant__ TmaMaps maps, GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kMaxStageBytes);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOutOffset + kEpiWarps * kStageOutBytes);
   // bars: full[kStages], empty[kStages], acc_full, acc_empty, drain, sf_full[kStages], sf_free[kScaleBufs],
   // sf_drain[kCopiers]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 3 + kScaleBufs + kCopiers);
@@ -465,6 +487,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int col_half = (warp - 2) >> 2;  // columns [128*col_half, 128*col_half + 128)
     const int r_local = quarter * 32 + lane;
     const uint32_t acc_empty_leader = map_to_rank(acc_empty, 0);
+    const uint32_t out_smem = smem0 + kOutOffset + (warp - 2) * kStageOutBytes;
     uint32_t acc_phase = 0;
     const float s_w = p.tensor_scale[0];
     for (int tile = pair; tile < num_tiles; tile += num_pairs) {
@@ -527,25 +550,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+        // Write this warp's 32 x 128 block with bulk tensor stores (coalesced; rows >= T and
+        // columns >= N clipped by the tensor map) through a 2 KB staging box of 32 x 32, in
+        // 64-byte-swizzled rows: 16-byte unit u of row r at u ^ ((r / 2) % 4), conflict-free.
+        const int row0 = m0 + quarter * 32;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const int col = col0 + 32 * c;
-          if (!row_ok || col >= p.N) continue;
-          uint16_t *dst = reinterpret_cast<uint16_t *>(p.y) + (size_t)row * p.N + col;
-          if (col + 32 <= p.N) {
+          if (lane == 0) bulk_wait_read();  // the previous box has been read out of the buffer
+          __syncwarp();
 #pragma unroll
-            for (int i = 0; i < 16; i += 4)
-              *reinterpret_cast<uint4 *>(dst + 2 * i) =
-                  make_uint4(packed[c][i], packed[c][i + 1], packed[c][i + 2], packed[c][i + 3]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (col + 2 * i < p.N) *reinterpret_cast<uint32_t *>(dst + 2 * i) = packed[c][i];
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t dst = out_smem + lane * 64 + ((u ^ ((lane >> 1) & 3)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(packed[c][4 * u]),
+                         "r"(packed[c][4 * u + 1]), "r"(packed[c][4 * u + 2]), "r"(packed[c][4 * u + 3])
+                         : "memory");
+          }
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            if (row0 < p.T && col0 + 32 * c < p.N) tma_store_2d(&maps.y, out_smem, col0 + 32 * c, row0);
+            bulk_commit();
           }
         }
       }
       acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();  // the output stores have completed before the CTA exits
   }
 
   else {
@@ -710,7 +740,21 @@ cudaError_t launch_gemm(const GemmParams &p, cudaStream_t st, const char **why) 
   const uint64_t ks = (uint64_t)p.K / BK;
   const uint64_t a_rows = (uint64_t)(p.T_pad / 128) * ks * (A.bytes / 1024);
   const uint64_t w_rows = (uint64_t)(p.N_pad / 128) * ks * (W.bytes / 1024);
-  if (!cache.get(&maps.act, p.a_tiles, a_rows, A.bytes / 1024) || !cache.get(&maps.w, p.w_tiles, w_rows, W.bytes / 1024)) {
+  bool y_ok = true;
+  if (!p.out_f32) {
+    auto fn = encode_fn();
+    cuuint64_t dims[2] = {(cuuint64_t)p.N, (cuuint64_t)p.T};
+    cuuint64_t strides[1] = {(cuuint64_t)p.N * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    y_ok = fn && fn(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.y, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  } else {
+    memset(&maps.y, 0, sizeof maps.y);
+  }
+  if (!y_ok || !cache.get(&maps.act, p.a_tiles, a_rows, A.bytes / 1024) ||
+      !cache.get(&maps.w, p.w_tiles, w_rows, W.bytes / 1024)) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or operand layout rejected)";
     return cudaErrorInvalidValue;
   }
