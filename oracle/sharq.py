@@ -254,6 +254,77 @@ def prepare(x, gamma, eps: float, n: int, m: int, unit: int, fmt: str) -> dict:
                 sp_deq=sp_deq, resid=resid, n=n, m=m, unit=unit, fmt=fmt)
 
 
+# --------------------------------------------------------------------------------------
+# SwiGLU fused into the preparation operator (down-projection input)
+# --------------------------------------------------------------------------------------
+# The abstract's fused preparation kernel absorbs the steps in front of the quantizer into
+# one operator; for a down projection that step is the gated activation x = SiLU(g) * u of
+# the gate/up projection's output [g | u]. Reading (the pages give no formula): the
+# activation the unfused pipeline hands to the down projection is bf16, so
+#   x = bf16_RNE(fp32(silu(g) * u)),  silu(g) = fp32(g * sigma(g)),
+#   sigma(g) = 1 / (1 + e) for g >= 0 and e / (1 + e) for g < 0, with e = exp(-|g|),
+# each step a float32 round-to-nearest operation (division correctly rounded). exp is
+# evaluated by range reduction with Cody and Waite's two-part ln 2 (W. J. Cody and W. Waite,
+# "Software Manual for the Elementary Functions", 1980) and a Taylor polynomial:
+#   a = |g|; t = fp32(a * log2(e)); t >= 126 gives e = 0 (below the normal range);
+#   n = rint(t); r = fp32(fp32(a - fp32(n * LN2_HI)) - fp32(n * LN2_LO)), |r| <~ ln2 / 2
+#   (n * LN2_HI is exact: LN2_HI has 15 significant bits, n at most 7);
+#   e^-r by Horner on the Taylor coefficients 1/k!, k = 7 .. 0, at -r, one rounding per
+#   multiply and per add (no fused multiply-add); e = fp32(p * 2^-n).
+# Written as separate correctly rounded float32 operations, the CUDA kernel reproduces
+# every bit of it.
+_LOG2E = F32(1.4426950408889634)
+_LN2_HI = F32(0.693145751953125)            # 0x3F317200
+_LN2_LO = F32(0.6931471805599453 - 0.693145751953125)
+_EXP_TAYLOR = [F32(1.0 / np.prod(np.arange(1, k + 1, dtype=np.float64))) for k in range(8)]
+
+
+def exp_neg_abs(g) -> np.ndarray:
+    """exp(-|g|) in float32: Cody-Waite reduction to r in [-ln2/2, ln2/2] plus degree-7 Taylor."""
+    a = np.abs(np.asarray(g, dtype=F32))
+    with np.errstate(over="ignore", invalid="ignore"):  # |g| beyond the range: masked at the end
+        t = (a * _LOG2E).astype(F32)
+        n = np.rint(np.minimum(t, F32(126.0))).astype(F32)       # 0 .. 126, ties to even
+        r = ((a - (n * _LN2_HI).astype(F32)).astype(F32) - (n * _LN2_LO).astype(F32)).astype(F32)
+        x = (-r).astype(F32)
+        p = np.full_like(x, _EXP_TAYLOR[7])
+        for k in range(6, -1, -1):
+            p = ((p * x).astype(F32) + _EXP_TAYLOR[k]).astype(F32)
+        scale = np.ldexp(F32(1.0), -n.astype(np.int32)).astype(F32)  # 2^-n, exact
+        e = (p * scale).astype(F32)
+    return np.where(t >= F32(126.0), F32(0.0), e).astype(F32)
+
+
+def silu(g) -> np.ndarray:
+    """SiLU(g) = g * sigmoid(g) in float32 (reading above)."""
+    g = np.asarray(g, dtype=F32)
+    e = exp_neg_abs(g)
+    den = (F32(1.0) + e).astype(F32)
+    num = np.where(g >= F32(0.0), F32(1.0), e).astype(F32)
+    sigma = (num / den).astype(F32)
+    return (g * sigma).astype(F32)
+
+
+def round_bf16(v) -> np.ndarray:
+    """float32 -> nearest bf16 (ties to even), returned as float32 values."""
+    b = np.ascontiguousarray(v, dtype=F32).view(np.uint32).astype(np.uint64)
+    r = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(F32)
+
+
+def swiglu(gate_up) -> np.ndarray:
+    """x [T, K] = bf16_RNE(fp32(silu(g) * u)) from gate_up [T, 2K] = [g | u]."""
+    gu = np.asarray(gate_up, dtype=F32)
+    K = gu.shape[1] // 2
+    prod = (silu(gu[:, :K]) * gu[:, K:]).astype(F32)
+    return round_bf16(prod)
+
+
+def prepare_swiglu(gate_up, n: int, m: int, unit: int, fmt: str) -> dict:
+    """The preparation operator on the gated activation of a down projection (no RMSNorm)."""
+    return prepare(swiglu(gate_up), None, 0.0, n, m, unit, fmt)
+
+
 def quantize_dense(x, gamma, eps: float, fmt: str) -> dict:
     """The plain dense FP4 activation quantizer (the README's "NVFP4: dense FP4 baseline" mode).
 

@@ -73,6 +73,12 @@ def swiglu_activations(rng, T: int, K: int) -> np.ndarray:
     return f32_to_bf16_bits(silu * u)
 
 
+def gate_up_activations(rng, T: int, K: int) -> np.ndarray:
+    """A gate/up projection's output [T, 2K] = [g | u] in bf16, g, u ~ N(0, 1) (the input of a
+    down projection whose preparation fuses the gated activation)."""
+    return f32_to_bf16_bits(rng.standard_normal((T, 2 * K), dtype=np.float32))
+
+
 def rms_gamma(rng, K: int) -> np.ndarray:
     return f32_to_bf16_bits(rng.uniform(0.5, 1.5, size=K).astype(np.float32))
 
@@ -110,6 +116,13 @@ def llama_down(seed: int = 2, T: int = 4096) -> Linear:
     rng = np.random.default_rng(seed + 100)
     K, N = 14336, 4096
     return Linear(f"llama31_8b_down_{T}x{K}x{N}", swiglu_activations(rng, T, K), None, weight(rng, N, K))
+
+
+def llama_down_gate_up(seed: int = 2, T: int = 2048) -> tuple[np.ndarray, np.ndarray]:
+    """Llama-3.1-8B down projection fed by its gate/up output: ([T, 2*14336] bf16, W [4096, 14336])."""
+    rng = np.random.default_rng(seed + 300)
+    K, N = 14336, 4096
+    return gate_up_activations(rng, T, K), weight(rng, N, K)
 
 
 QWEN_LINEARS = {  # name: (K, N, fused RMSNorm)
