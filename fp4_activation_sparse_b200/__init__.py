@@ -11,6 +11,7 @@ Quantization for LLM Inference", Abstract):
   sharq_pack_weight  - one FP4 weight payload with sparse-path and dense-path scale views
   sharq_prepare      - the fused preparation operator (RMSNorm, N:M mask, FP4 backbone,
                        residual against the quantized backbone, dense FP4 residual)
+  sharq_prepare_swiglu - the same operator on a down projection's gated input SiLU(g)*u
   sharq_linear       - sparse FP4 GEMM + dense FP4 GEMM into one output
 and the library's dense FP4 baseline (the README's "NVFP4" mode):
   sharq_quantize_dense, sharq_linear_dense.
@@ -63,6 +64,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sharq_wpack_buffer_sizes": (S, [I, I, I, ctypes.POINTER(S)]),
         "sharq_pack_weight": (I, [P, I, I, I, ctypes.POINTER(_WPack), P]),
         "sharq_prepare": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P]),
+        "sharq_prepare_swiglu": (I, [P, I, I, I, I, I, I, ctypes.POINTER(_Prep), P]),
         "sharq_linear": (I, [ctypes.POINTER(_Prep), ctypes.POINTER(_WPack), P, I, P]),
         "sharq_quantize_dense": (I, [P, I, I, P, F, I, P, P, P]),
         "sharq_linear_dense": (I, [P, P, I, I, ctypes.POINTER(_WPack), P, I, P]),
@@ -214,6 +216,21 @@ def sharq_prepare(x: torch.Tensor, gamma: torch.Tensor | None = None, eps: float
     st = out.struct()
     _check(lib.sharq_prepare(_ptr(x), tokens, k, _ptr(gamma), ctypes.c_float(eps), nm_n, nm_m, unit, _fmt(fmt),
                              ctypes.byref(st), _stream(stream)))
+    return out
+
+
+def sharq_prepare_swiglu(gate_up: torch.Tensor, nm_n: int = 2, nm_m: int = 4, unit: int = UNIT_PAIR,
+                         fmt="nvfp4", out: Prep | None = None, stream=None) -> Prep:
+    """The preparation operator on a down projection's gated input x = SiLU(g) * u, formed in
+    registers from the gate/up output [tokens, 2k] = [g | u] (bf16, device)."""
+    assert gate_up.dtype == torch.bfloat16 and gate_up.is_cuda and gate_up.is_contiguous()
+    tokens, k2 = gate_up.shape
+    assert k2 % 2 == 0
+    k = k2 // 2
+    out = out or alloc_prep(tokens, k, nm_n, nm_m, unit, fmt, gate_up.device)
+    st = out.struct()
+    _check(lib.sharq_prepare_swiglu(_ptr(gate_up), tokens, k, nm_n, nm_m, unit, _fmt(fmt), ctypes.byref(st),
+                                    _stream(stream)))
     return out
 
 

@@ -111,7 +111,7 @@ int sharq_pack_weight(const void *w, int n_out, int k, int fmt, sharq_wpack *out
 }
 
 static int prepare_common(const void *x, int tokens, int k, const void *gamma, float eps, int fmt, bool dense,
-                          int unit, uint8_t *tiles, float *row_scale, cudaStream_t st) {
+                          int unit, uint8_t *tiles, float *row_scale, cudaStream_t st, bool swiglu = false) {
   if (!x) return fail(SHARQ_ERR_INVALID_ARG, "x is null");
   if (!valid_fmt(fmt)) return fail(SHARQ_ERR_INVALID_ARG, "unknown fmt %d", fmt);
   if (int s = check_shape(tokens, k, "tokens")) return s;
@@ -123,6 +123,7 @@ static int prepare_common(const void *x, int tokens, int k, const void *gamma, f
   if (gamma && !(eps >= 0.f)) return fail(SHARQ_ERR_INVALID_ARG, "eps must be >= 0");
   sharq::PrepParams p;
   p.x = static_cast<const uint16_t *>(x);
+  p.x_stride = swiglu ? 2 * k : k;
   p.gamma = static_cast<const uint16_t *>(gamma);
   p.eps = eps;
   p.T = tokens;
@@ -130,8 +131,9 @@ static int prepare_common(const void *x, int tokens, int k, const void *gamma, f
   p.T_pad = sharq::round_up(tokens, 256);
   p.tiles = tiles;
   p.row_scale = row_scale;
-  cudaError_t e = sharq::launch_prep(p, fmt, unit, gamma != nullptr, dense, st);
-  if (e != cudaSuccess) return cuda_fail(e, dense ? "sharq_quantize_dense" : "sharq_prepare");
+  cudaError_t e = sharq::launch_prep(p, fmt, unit, gamma != nullptr, dense, swiglu, st);
+  if (e != cudaSuccess)
+    return cuda_fail(e, dense ? "sharq_quantize_dense" : swiglu ? "sharq_prepare_swiglu" : "sharq_prepare");
   g_err[0] = 0;
   return SHARQ_OK;
 }
@@ -142,6 +144,24 @@ int sharq_prepare(const void *x, int tokens, int k, const void *gamma, float eps
   if (int s = check_pattern(nm_n, nm_m, unit)) return s;
   int s = prepare_common(x, tokens, k, gamma, eps, fmt, false, unit, static_cast<uint8_t *>(out->tiles),
                          out->row_scale, static_cast<cudaStream_t>(stream));
+  if (s == SHARQ_OK) {
+    out->tokens = tokens;
+    out->k = k;
+    out->nm_n = nm_n;
+    out->nm_m = nm_m;
+    out->unit = unit;
+    out->fmt = fmt;
+  }
+  return s;
+}
+
+int sharq_prepare_swiglu(const void *gate_up, int tokens, int k, int nm_n, int nm_m, int unit, int fmt,
+                         sharq_prep *out, void *stream) {
+  if (!out) return fail(SHARQ_ERR_INVALID_ARG, "output struct is null");
+  if (int s = check_pattern(nm_n, nm_m, unit)) return s;
+  if (tokens > 0 && (long long)tokens * 2 * k > (1ll << 40)) return fail(SHARQ_ERR_INVALID_ARG, "tensor too large");
+  int s = prepare_common(gate_up, tokens, k, nullptr, 0.f, fmt, false, unit, static_cast<uint8_t *>(out->tiles),
+                         out->row_scale, static_cast<cudaStream_t>(stream), true);
   if (s == SHARQ_OK) {
     out->tokens = tokens;
     out->k = k;

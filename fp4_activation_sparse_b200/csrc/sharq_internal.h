@@ -45,8 +45,9 @@ __host__ __device__ constexpr WTile w_tile(int fmt) {
 __host__ __device__ constexpr int atom_pos(int r, int s) { return (s >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (s & 3); }
 
 struct PrepParams {
-  const uint16_t *x;      // [T][K] bf16
+  const uint16_t *x;      // [T][x_stride] bf16: the activation, or [g | u] for the gated form
   const uint16_t *gamma;  // [K] bf16 or null
+  int x_stride;           // elements per input row: K, or 2K for the gated form
   float eps;
   int T, K, T_pad;
   int KS;  // 256-K steps per row
@@ -73,7 +74,7 @@ struct GemmParams {
   long long wait_limit;
 };
 
-cudaError_t launch_prep(PrepParams p, int fmt, int unit, bool norm, bool dense, cudaStream_t st);
+cudaError_t launch_prep(PrepParams p, int fmt, int unit, bool norm, bool dense, bool swiglu, cudaStream_t st);
 cudaError_t launch_pack(PackParams p, int fmt, cudaStream_t st);
 cudaError_t launch_gemm(const GemmParams &p, cudaStream_t st, const char **why);
 cudaError_t read_and_clear_device_status(int *status, cudaStream_t st);

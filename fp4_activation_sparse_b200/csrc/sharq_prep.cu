@@ -83,6 +83,51 @@ __device__ __forceinline__ double add_squares(uint32_t w, double ss) {
   return __fma_rn(hi, hi, __fma_rn(lo, lo, ss));
 }
 
+// ---------------------------------------------------------------- gated activation
+// x = bf16_RNE(fp32(silu(g) * u)) with silu(g) = fp32(g * sigma(g)), sigma(g) = 1/(1+e) for
+// g >= 0 and e/(1+e) for g < 0, e = exp(-|g|) -- the down projection's input computed inside
+// the preparation operator. exp by range reduction with Cody and Waite's two-part ln 2 and a
+// degree-7 Taylor polynomial of e^x on |x| <= ln2/2 (W. J. Cody and W. Waite, "Software
+// Manual for the Elementary Functions", 1980): every step a separate round-to-nearest
+// float32 operation, the division correctly rounded, no fused multiply-add, so the result
+// is a fixed function of g (|g| log2 e >= 126 gives e = 0).
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2Hi = 0.693145751953125f;  // 15 significant bits: n * kLn2Hi is exact for n <= 126
+constexpr float kLn2Lo = (float)(0.6931471805599453 - 0.693145751953125);
+
+__device__ __forceinline__ float exp_neg_abs(float g) {
+  const float a = fabsf(g);
+  const float t = __fmul_rn(a, kLog2e);
+  const float n = rintf(fminf(t, 126.f));
+  const float r = __fsub_rn(__fsub_rn(a, __fmul_rn(n, kLn2Hi)), __fmul_rn(n, kLn2Lo));
+  const float x = -r;
+  float q = (float)(1.0 / 5040.0);
+  q = __fadd_rn(__fmul_rn(q, x), (float)(1.0 / 720.0));
+  q = __fadd_rn(__fmul_rn(q, x), (float)(1.0 / 120.0));
+  q = __fadd_rn(__fmul_rn(q, x), (float)(1.0 / 24.0));
+  q = __fadd_rn(__fmul_rn(q, x), (float)(1.0 / 6.0));
+  q = __fadd_rn(__fmul_rn(q, x), 0.5f);
+  q = __fadd_rn(__fmul_rn(q, x), 1.f);
+  q = __fadd_rn(__fmul_rn(q, x), 1.f);
+  const float e = __fmul_rn(q, __int_as_float((127 - (int)n) << 23));  // * 2^-n, exact scale
+  return t >= 126.f ? 0.f : e;
+}
+
+__device__ __forceinline__ float gated(float g, float u) {
+  const float e = exp_neg_abs(g);
+  const float sigma = __fdiv_rn(g >= 0.f ? 1.f : e, __fadd_rn(1.f, e));
+  return __fmul_rn(__fmul_rn(g, sigma), u);
+}
+
+// 16 gated activations from a 256-bit word group of g and one of u, as packed bf16 (RNE)
+__device__ __forceinline__ void gated16(const uint32_t (&g)[8], const uint32_t (&u)[8], uint32_t (&x)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(gated(bf16lo(g[i]), bf16lo(u[i])), gated(bf16hi(g[i]), bf16hi(u[i])));
+    x[i] = *reinterpret_cast<const uint32_t *>(&h);
+  }
+}
+
 __device__ __forceinline__ void unpack16(const uint32_t (&w)[8], float *v) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -366,7 +411,7 @@ __device__ __forceinline__ void row_scales(int fmt, float amax, float &s_x, floa
 }
 
 // ---------------------------------------------------------------- kernel
-template <int FMT, int UNIT, bool NORM, bool DENSE>
+template <int FMT, int UNIT, bool NORM, bool DENSE, bool SWIGLU>
 __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   extern __shared__ float4 gamma_smem4[];  // NORM: the RMSNorm weight as float32 (K rounded up to 512)
   __shared__ double sm_d[64];
@@ -384,7 +429,15 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
 #pragma unroll
   for (int i = 0; i < kMaxDP; ++i) {
     const int dp = i * stride + wt * 32 + lane;
-    if (live_row && dp < ndp_row) ld256(p.x + (size_t)row * p.K + (size_t)dp * 16, xr[i]);
+    if (live_row && dp < ndp_row) {
+      const uint16_t *src = p.x + (size_t)row * p.x_stride + (size_t)dp * 16;
+      ld256(src, xr[i]);
+      if (SWIGLU) {  // xr holds g; u sits K columns further
+        uint32_t u[8];
+        ld256(src + p.K, u);
+        gated16(xr[i], u, xr[i]);
+      }
+    }
   }
 
   float rstd = 1.f;
@@ -460,7 +513,7 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   if (live_row && wt == 0 && lane == 0) p.row_scale[row] = s_x;
 }
 
-template <int FMT, int UNIT, bool NORM, bool DENSE>
+template <int FMT, int UNIT, bool NORM, bool DENSE, bool SWIGLU = false>
 cudaError_t launch_t(const PrepParams &p, cudaStream_t st) {
   const int W = p.TS;
   const int teams = W >= 8 ? 1 : 8 / W;
@@ -477,12 +530,12 @@ cudaError_t launch_t(const PrepParams &p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [dev] {
-      err[dev] = cudaFuncSetAttribute(prep_kernel<FMT, UNIT, NORM, DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      err[dev] = cudaFuncSetAttribute(prep_kernel<FMT, UNIT, NORM, DENSE, SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       32768 * (int)sizeof(float));
     });
     if (err[dev] != cudaSuccess) return err[dev];
   }
-  prep_kernel<FMT, UNIT, NORM, DENSE><<<grid, block, smem, st>>>(p);
+  prep_kernel<FMT, UNIT, NORM, DENSE, SWIGLU><<<grid, block, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -496,12 +549,17 @@ cudaError_t launch_n(const PrepParams &p, bool norm, cudaStream_t st) {
 // Warps per row: each lane holds at most kMaxDP double pieces (16 elements each).
 int prep_team_warps(int k) { return (k / 16 + 32 * kMaxDP - 1) / (32 * kMaxDP); }
 
-cudaError_t launch_prep(PrepParams p, int fmt, int unit, bool norm, bool dense, cudaStream_t st) {
+cudaError_t launch_prep(PrepParams p, int fmt, int unit, bool norm, bool dense, bool swiglu, cudaStream_t st) {
   p.KS = p.K / 256;
   p.TS = prep_team_warps(p.K);
   if (p.TS > 8) return cudaErrorInvalidValue;  // k > 32768: outside the supported range
   if (dense) {
     return fmt == kFmtNV ? launch_n<kFmtNV, 2, true>(p, norm, st) : launch_n<kFmtMX, 2, true>(p, norm, st);
+  }
+  if (swiglu) {  // the gated activation of a down projection (no normalization)
+    if (fmt == kFmtNV)
+      return unit == 2 ? launch_t<kFmtNV, 2, false, false, true>(p, st) : launch_t<kFmtNV, 1, false, false, true>(p, st);
+    return unit == 2 ? launch_t<kFmtMX, 2, false, false, true>(p, st) : launch_t<kFmtMX, 1, false, false, true>(p, st);
   }
   if (fmt == kFmtNV)
     return unit == 2 ? launch_n<kFmtNV, 2, false>(p, norm, st) : launch_n<kFmtNV, 1, false>(p, norm, st);

@@ -153,6 +153,20 @@ int sharq_prepare(const void *x_bf16_dev, int tokens, int k, const void *gamma_b
                   float eps, int nm_n, int nm_m, int unit, int fmt, sharq_prep *out,
                   void *stream);
 
+/* The preparation operator fed by a gate/up projection's output (one launch): the down
+ * projection's input x = SiLU(g) * u is formed in registers from [g | u] and prepared as
+ * by sharq_prepare without normalization, so x never goes through memory. The abstract's
+ * fused preparation kernel "absorbs" the steps in front of the quantizer into one operator.
+ *   gate_up_bf16_dev  [tokens][2k] row-major bf16: g in columns [0, k), u in [k, 2k);
+ *                     32-byte aligned
+ *   x = bf16(fp32(silu(g) * u)) rounded to nearest even, silu(g) = g * sigma(g) in float32
+ *   with sigma(g) = 1/(1+e) (g >= 0) or e/(1+e) (g < 0), e = exp(-|g|) evaluated by Cody-Waite
+ *   range reduction and a degree-7 Taylor polynomial in correctly rounded float32 steps
+ *   (|g| * log2(e) >= 126 gives e = 0); the division is correctly rounded.
+ * Output, pattern, formats and errors as sharq_prepare. */
+int sharq_prepare_swiglu(const void *gate_up_bf16_dev, int tokens, int k, int nm_n, int nm_m,
+                         int unit, int fmt, sharq_prep *out, void *stream);
+
 /* The SharQ linear layer (one launch): Y = s_x * s_w * (A_sp (*) W^T + A_res . W^T),
  * the structured-sparse block-scaled FP4 MMA on the backbone and the dense one on
  * the residual accumulating into one tensor-memory accumulator, then one epilogue.
