@@ -323,6 +323,31 @@ def run_sharq(args, rank, world, local):
     t_dl = graph_time(capture(lambda st: S.sharq_linear_dense(q, wps[0], y=yd, stream=st)), 1)
     del w_bf16
 
+    # ---- the gated-activation preparation (down projection fed by its gate/up output):
+    # fused kernel vs the unfused pipeline (torch SiLU * up in bf16, then the preparation)
+    gu_bits, _ = wl.llama_down_gate_up(seed=replica_seed(rank), T=T)
+    Kd = gu_bits.shape[1] // 2
+    n_gu = max(2, int(np.ceil(2 * L2_BYTES / (T * Kd * 4))))  # rotate inputs beyond L2
+    gus = [to_dev(gu_bits) for _ in range(n_gu)]
+    del gu_bits
+    p_sw = S.sharq_prepare_swiglu(gus[0])
+    x_sw = torch.empty(T, Kd, dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    t_sw = graph_time(capture(lambda st: [S.sharq_prepare_swiglu(g_, out=p_sw, stream=st) for g_ in gus]), n_gu)
+
+    def unfused(st):
+        for g_ in gus:
+            torch.mul(torch.nn.functional.silu(g_[:, :Kd]), g_[:, Kd:], out=x_sw)
+            S.sharq_prepare(x_sw, None, 0.0, out=p_sw, stream=st)
+
+    with torch.cuda.stream(cap):
+        unfused(cap)
+    torch.cuda.synchronize()
+    t_unf = graph_time(capture(unfused), n_gu)
+    sw_bytes = T * Kd * (4 + PREP_BYTES_PER_ELEM - 2) + T * 4
+    sw_gbs = sw_bytes / (t_sw / 1e3) / 1e9
+    del gus
+
     # ---- end to end through the public API with host buffers: every step copies its input
     # from pinned host memory and its output back. Copies run on their own streams and overlap
     # the previous/next step's kernels (double-buffered device and host buffers).
@@ -404,6 +429,10 @@ def run_sharq(args, rank, world, local):
                       "dense_nvfp4_quantize_us": t_dq * 1e3, "dense_nvfp4_gemm_us": t_dl * 1e3},
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * K * 2,
                 "d2h_bytes_per_step": T * N * 2},
+        "next": {"swiglu_prep": {
+            "workload": f"llama31_8b_down_from_gate_up T={T} K={Kd} nvfp4 2:4-pairs (x = SiLU(g)*u in the kernel)",
+            "t_us": t_sw * 1e3, "achieved_gbs": sw_gbs, "bound": "hbm", "peak_gbs": hbm_peak,
+            "frac": sw_gbs / hbm_peak, "unfused_torch_swiglu_plus_prep_us": t_unf * 1e3}},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "device_status": status,
