@@ -144,15 +144,19 @@ def scatter_kept(stored: np.ndarray, idx: np.ndarray, k: int, m: int, unit: int)
 # --------------------------------------------------------------------------------------
 # steps a3 / a5: block quantization
 # --------------------------------------------------------------------------------------
-def row_scale(xh: np.ndarray, fmt: str):
-    """Per-row second-level scale s_x and its encode factor g_x = 1/(6*s_x) (NVFP4).
+def row_scale(xh: np.ndarray, fmt: str, per_tensor: bool = False):
+    """Second-level scale s_x and its encode factor g_x = 1/(6*s_x) (NVFP4), one per row.
 
-    MXFP4 has no second-level scale: s_x = 1, g_x unused (returned as 1).
+    per_tensor: one scale for the whole tensor (amax over every row), repeated per row -- the
+    stricter reading of NVFP4's "fp32 tensor scale". MXFP4 has no second-level scale:
+    s_x = 1, g_x unused (returned as 1).
     """
     T = xh.shape[0]
     if fmt == MXFP4:
         return np.ones(T, dtype=F32), np.ones(T, dtype=F32)
     amax = np.abs(xh).max(axis=1).astype(F32)
+    if per_tensor:
+        amax = np.full(T, amax.max() if T else F32(0.0), dtype=F32)
     zero = amax == 0
     safe = np.where(zero, F32(1.0), amax).astype(F32)
     s_x = np.where(zero, F32(1.0), safe / _E4M3_TIMES_E2M1_MAX).astype(F32)
@@ -227,7 +231,7 @@ def _quantize(vals2d: np.ndarray, fmt: str, s_x, g_x):
 # --------------------------------------------------------------------------------------
 # the preparation operator (steps a1-a5)
 # --------------------------------------------------------------------------------------
-def prepare(x, gamma, eps: float, n: int, m: int, unit: int, fmt: str) -> dict:
+def prepare(x, gamma, eps: float, n: int, m: int, unit: int, fmt: str, per_tensor: bool = False) -> dict:
     """SharQ's fused preparation operator, written out step by step.
 
     Abstract: mask -> backbone -> "quantizes it to FP4" -> "defines a dense
@@ -238,11 +242,14 @@ def prepare(x, gamma, eps: float, n: int, m: int, unit: int, fmt: str) -> dict:
       xh [T,K] f32, idx [T,G,n], sp_codes [T,K*n/m] u8, sp_scales [T,nb_sp] u8,
       res_codes [T,K] u8, res_scales [T,nb_res] u8, row_scale [T] f32,
       sp_deq [T,K*n/m] f32, resid [T,K] f32.
+
+    per_tensor: one second-level scale for the whole activation tensor instead of one per
+    row (NVFP4; the variant of the reading "fp32 tensor scale"), shared by both paths.
     """
     x = np.asarray(x, dtype=F32)
     T, K = x.shape
     xh = rmsnorm(x, gamma, eps)
-    s_x, g_x = row_scale(xh, fmt)
+    s_x, g_x = row_scale(xh, fmt, per_tensor)
     idx = nm_select(xh, n, m, unit)
     stored = gather_kept(xh, idx, m, unit)
     sp_codes, sp_scales, sp_deq = _quantize(stored, fmt, s_x, g_x)

@@ -298,3 +298,37 @@ def test_sharq_error_below_dense_nvfp4_on_outlier_inputs():
         e_sharq = np.linalg.norm(O.linear(p, wp) - ref)
         e_dense = np.linalg.norm(O.linear_dense(q, wp) - ref)
         assert e_sharq < e_dense
+
+
+# ---------------------------------------------------------------- per-tensor activation scale
+def test_per_tensor_scale_single_row_equals_per_row():
+    """With one token row the tensor amax is the row amax: both readings coincide."""
+    x = wl.bf16_bits_to_f32(wl.outlier_activations(np.random.default_rng(21), 1, 512, 4, 20.0, 100.0, 0.5))
+    a = O.prepare(x, None, 1e-6, 2, 4, 2, O.NVFP4)
+    b = O.prepare(x, None, 1e-6, 2, 4, 2, O.NVFP4, per_tensor=True)
+    for k in ("sp_codes", "res_codes", "sp_scales", "res_scales", "row_scale", "idx"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_per_tensor_scale_is_the_largest_row_scale():
+    x = wl.bf16_bits_to_f32(wl.outlier_activations(np.random.default_rng(22), 32, 512, 4, 20.0, 100.0, 0.5))
+    a = O.prepare(x, None, 1e-6, 2, 4, 2, O.NVFP4)
+    b = O.prepare(x, None, 1e-6, 2, 4, 2, O.NVFP4, per_tensor=True)
+    assert np.all(b["row_scale"] == a["row_scale"].max())
+    # the row holding the tensor amax is quantized exactly as with its own row scale
+    r = int(np.argmax(a["row_scale"]))
+    for k in ("sp_codes", "res_codes", "sp_scales", "res_scales"):
+        assert np.array_equal(a[k][r], b[k][r]), k
+    # other rows use a larger scale: their block scales can only shrink
+    others = np.arange(32) != r
+    assert np.all(e4m3_decode(b["sp_scales"][others]) <= e4m3_decode(a["sp_scales"][others]))
+
+
+def test_per_tensor_scale_power_of_two_invariance():
+    """Scaling X by 2^k scales s_x by 2^k and leaves every code and block scale unchanged."""
+    x = wl.bf16_bits_to_f32(wl.outlier_activations(np.random.default_rng(23), 16, 256, 2, 20.0, 100.0, 0.5))
+    a = O.prepare(x, None, 1e-6, 2, 4, 2, O.NVFP4, per_tensor=True)
+    b = O.prepare(x * np.float32(8.0), None, 1e-6, 2, 4, 2, O.NVFP4, per_tensor=True)
+    for k in ("sp_codes", "res_codes", "sp_scales", "res_scales", "idx"):
+        assert np.array_equal(a[k], b[k]), k
+    assert np.array_equal(b["row_scale"], a["row_scale"] * np.float32(8.0))
