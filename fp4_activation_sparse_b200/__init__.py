@@ -12,6 +12,7 @@ Quantization for LLM Inference", Abstract):
   sharq_prepare      - the fused preparation operator (RMSNorm, N:M mask, FP4 backbone,
                        residual against the quantized backbone, dense FP4 residual)
   sharq_prepare_swiglu - the same operator on a down projection's gated input SiLU(g)*u
+  sharq_prepare_tensor_scale - the same operator with one NVFP4 second-level scale per tensor
   sharq_linear       - sparse FP4 GEMM + dense FP4 GEMM into one output
 and the library's dense FP4 baseline (the README's "NVFP4" mode):
   sharq_quantize_dense, sharq_linear_dense.
@@ -65,6 +66,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sharq_pack_weight": (I, [P, I, I, I, ctypes.POINTER(_WPack), P]),
         "sharq_prepare": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P]),
         "sharq_prepare_swiglu": (I, [P, I, I, I, I, I, I, ctypes.POINTER(_Prep), P]),
+        "sharq_prepare_tensor_scale": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P]),
         "sharq_linear": (I, [ctypes.POINTER(_Prep), ctypes.POINTER(_WPack), P, I, P]),
         "sharq_quantize_dense": (I, [P, I, I, P, F, I, P, P, P]),
         "sharq_linear_dense": (I, [P, P, I, I, ctypes.POINTER(_WPack), P, I, P]),
@@ -216,6 +218,22 @@ def sharq_prepare(x: torch.Tensor, gamma: torch.Tensor | None = None, eps: float
     st = out.struct()
     _check(lib.sharq_prepare(_ptr(x), tokens, k, _ptr(gamma), ctypes.c_float(eps), nm_n, nm_m, unit, _fmt(fmt),
                              ctypes.byref(st), _stream(stream)))
+    return out
+
+
+def sharq_prepare_tensor_scale(x: torch.Tensor, gamma: torch.Tensor | None = None, eps: float = 1e-6,
+                               nm_n: int = 2, nm_m: int = 4, unit: int = UNIT_PAIR, fmt="nvfp4",
+                               out: Prep | None = None, stream=None) -> Prep:
+    """sharq_prepare with one NVFP4 second-level scale for the whole tensor (every row_scale
+    entry holds it)."""
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous()
+    tokens, k = x.shape
+    if gamma is not None:
+        assert gamma.dtype == torch.bfloat16 and gamma.is_cuda and gamma.numel() == k
+    out = out or alloc_prep(tokens, k, nm_n, nm_m, unit, fmt, x.device)
+    st = out.struct()
+    _check(lib.sharq_prepare_tensor_scale(_ptr(x), tokens, k, _ptr(gamma), ctypes.c_float(eps), nm_n, nm_m, unit,
+                                          _fmt(fmt), ctypes.byref(st), _stream(stream)))
     return out
 
 

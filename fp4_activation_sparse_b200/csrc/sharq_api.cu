@@ -111,7 +111,8 @@ int sharq_pack_weight(const void *w, int n_out, int k, int fmt, sharq_wpack *out
 }
 
 static int prepare_common(const void *x, int tokens, int k, const void *gamma, float eps, int fmt, bool dense,
-                          int unit, uint8_t *tiles, float *row_scale, cudaStream_t st, bool swiglu = false) {
+                          int unit, uint8_t *tiles, float *row_scale, cudaStream_t st, bool swiglu = false,
+                          bool per_tensor = false) {
   if (!x) return fail(SHARQ_ERR_INVALID_ARG, "x is null");
   if (!valid_fmt(fmt)) return fail(SHARQ_ERR_INVALID_ARG, "unknown fmt %d", fmt);
   if (int s = check_shape(tokens, k, "tokens")) return s;
@@ -131,7 +132,8 @@ static int prepare_common(const void *x, int tokens, int k, const void *gamma, f
   p.T_pad = sharq::round_up(tokens, 256);
   p.tiles = tiles;
   p.row_scale = row_scale;
-  cudaError_t e = sharq::launch_prep(p, fmt, unit, gamma != nullptr, dense, swiglu, st);
+  cudaError_t e = per_tensor && fmt == SHARQ_NVFP4 ? sharq::launch_prep_tensor_scale(p, unit, gamma != nullptr, st)
+                                                   : sharq::launch_prep(p, fmt, unit, gamma != nullptr, dense, swiglu, st);
   if (e != cudaSuccess)
     return cuda_fail(e, dense ? "sharq_quantize_dense" : swiglu ? "sharq_prepare_swiglu" : "sharq_prepare");
   g_err[0] = 0;
@@ -144,6 +146,23 @@ int sharq_prepare(const void *x, int tokens, int k, const void *gamma, float eps
   if (int s = check_pattern(nm_n, nm_m, unit)) return s;
   int s = prepare_common(x, tokens, k, gamma, eps, fmt, false, unit, static_cast<uint8_t *>(out->tiles),
                          out->row_scale, static_cast<cudaStream_t>(stream));
+  if (s == SHARQ_OK) {
+    out->tokens = tokens;
+    out->k = k;
+    out->nm_n = nm_n;
+    out->nm_m = nm_m;
+    out->unit = unit;
+    out->fmt = fmt;
+  }
+  return s;
+}
+
+int sharq_prepare_tensor_scale(const void *x, int tokens, int k, const void *gamma, float eps, int nm_n, int nm_m,
+                               int unit, int fmt, sharq_prep *out, void *stream) {
+  if (!out) return fail(SHARQ_ERR_INVALID_ARG, "output struct is null");
+  if (int s = check_pattern(nm_n, nm_m, unit)) return s;
+  int s = prepare_common(x, tokens, k, gamma, eps, fmt, false, unit, static_cast<uint8_t *>(out->tiles),
+                         out->row_scale, static_cast<cudaStream_t>(stream), false, true);
   if (s == SHARQ_OK) {
     out->tokens = tokens;
     out->k = k;

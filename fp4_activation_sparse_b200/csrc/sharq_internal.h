@@ -75,6 +75,7 @@ struct GemmParams {
 };
 
 cudaError_t launch_prep(PrepParams p, int fmt, int unit, bool norm, bool dense, bool swiglu, cudaStream_t st);
+cudaError_t launch_prep_tensor_scale(PrepParams p, int unit, bool norm, cudaStream_t st);
 cudaError_t launch_pack(PackParams p, int fmt, cudaStream_t st);
 cudaError_t launch_gemm(const GemmParams &p, cudaStream_t st, const char **why);
 cudaError_t read_and_clear_device_status(int *status, cudaStream_t st);

@@ -411,7 +411,14 @@ __device__ __forceinline__ void row_scales(int fmt, float amax, float &s_x, floa
 }
 
 // ---------------------------------------------------------------- kernel
-template <int FMT, int UNIT, bool NORM, bool DENSE, bool SWIGLU>
+// Kernel modes. kRow: one second-level scale per row (written to row_scale). kSwiglu: as kRow,
+// the input formed as SiLU(g)*u from [g | u]. kAmax: only the row amax of xh, max-reduced into
+// row_scale[0] (float bits of a non-negative value order like unsigned integers). kTensor: the
+// second-level scale from the tensor amax left in row_scale[0] by kAmax; row_scale itself is
+// written afterwards by fill_row_scale (blocks still read row_scale[0] while others finish).
+constexpr int kRow = 0, kSwiglu = 1, kAmax = 2, kTensor = 3;
+
+template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE>
 __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   extern __shared__ float4 gamma_smem4[];  // NORM: the RMSNorm weight as float32 (K rounded up to 512)
   __shared__ double sm_d[64];
@@ -432,7 +439,7 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
     if (live_row && dp < ndp_row) {
       const uint16_t *src = p.x + (size_t)row * p.x_stride + (size_t)dp * 16;
       ld256(src, xr[i]);
-      if (SWIGLU) {  // xr holds g; u sits K columns further
+      if (MODE == kSwiglu) {  // xr holds g; u sits K columns further
         uint32_t u[8];
         ld256(src + p.K, u);
         gated16(xr[i], u, xr[i]);
@@ -480,6 +487,11 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
     }
   }
   am = team_max(am, W, team, wt, sm_f);
+  if (MODE == kAmax) {
+    if (live_row && wt == 0 && lane == 0) atomicMax(reinterpret_cast<unsigned int *>(p.row_scale), __float_as_uint(am));
+    return;
+  }
+  if (MODE == kTensor) am = p.row_scale[0];  // the tensor amax (kAmax pass)
   float s_x, g_x;
   row_scales(FMT, am, s_x, g_x);
 
@@ -510,10 +522,23 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
       store16<FMT, UNIT, DENSE>(chunk, o, 0u, 0u, 0u, 0u, 0u, 0u);
     }
   }
-  if (live_row && wt == 0 && lane == 0) p.row_scale[row] = s_x;
+  if (MODE != kTensor && live_row && wt == 0 && lane == 0) p.row_scale[row] = s_x;
 }
 
-template <int FMT, int UNIT, bool NORM, bool DENSE, bool SWIGLU = false>
+// Per-tensor scale: every row's entry gets the NVFP4 scale of the tensor amax held in
+// row_scale[0] (one block; entry 0 is read before any is written).
+__global__ void __launch_bounds__(1024) fill_row_scale(float *row_scale, int T) {
+  __shared__ float s_x;
+  if (threadIdx.x == 0) {
+    float s, g;
+    row_scales(kFmtNV, row_scale[0], s, g);
+    s_x = s;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < T; i += blockDim.x) row_scale[i] = s_x;
+}
+
+template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE = kRow>
 cudaError_t launch_t(const PrepParams &p, cudaStream_t st) {
   const int W = p.TS;
   const int teams = W >= 8 ? 1 : 8 / W;
@@ -530,12 +555,12 @@ cudaError_t launch_t(const PrepParams &p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [dev] {
-      err[dev] = cudaFuncSetAttribute(prep_kernel<FMT, UNIT, NORM, DENSE, SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      err[dev] = cudaFuncSetAttribute(prep_kernel<FMT, UNIT, NORM, DENSE, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       32768 * (int)sizeof(float));
     });
     if (err[dev] != cudaSuccess) return err[dev];
   }
-  prep_kernel<FMT, UNIT, NORM, DENSE, SWIGLU><<<grid, block, smem, st>>>(p);
+  prep_kernel<FMT, UNIT, NORM, DENSE, MODE><<<grid, block, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -558,12 +583,32 @@ cudaError_t launch_prep(PrepParams p, int fmt, int unit, bool norm, bool dense, 
   }
   if (swiglu) {  // the gated activation of a down projection (no normalization)
     if (fmt == kFmtNV)
-      return unit == 2 ? launch_t<kFmtNV, 2, false, false, true>(p, st) : launch_t<kFmtNV, 1, false, false, true>(p, st);
-    return unit == 2 ? launch_t<kFmtMX, 2, false, false, true>(p, st) : launch_t<kFmtMX, 1, false, false, true>(p, st);
+      return unit == 2 ? launch_t<kFmtNV, 2, false, false, kSwiglu>(p, st)
+                       : launch_t<kFmtNV, 1, false, false, kSwiglu>(p, st);
+    return unit == 2 ? launch_t<kFmtMX, 2, false, false, kSwiglu>(p, st) : launch_t<kFmtMX, 1, false, false, kSwiglu>(p, st);
   }
   if (fmt == kFmtNV)
     return unit == 2 ? launch_n<kFmtNV, 2, false>(p, norm, st) : launch_n<kFmtNV, 1, false>(p, norm, st);
   return unit == 2 ? launch_n<kFmtMX, 2, false>(p, norm, st) : launch_n<kFmtMX, 1, false>(p, norm, st);
+}
+
+// NVFP4 with one second-level scale for the whole tensor: tensor amax (clear + one pass),
+// the preparation with that scale, then the per-row copies of the scale.
+cudaError_t launch_prep_tensor_scale(PrepParams p, int unit, bool norm, cudaStream_t st) {
+  p.KS = p.K / 256;
+  p.TS = prep_team_warps(p.K);
+  if (p.TS > 8) return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(p.row_scale, 0, sizeof(float), st);
+  if (e != cudaSuccess) return e;
+  e = norm ? launch_t<kFmtNV, 2, true, false, kAmax>(p, st) : launch_t<kFmtNV, 2, false, false, kAmax>(p, st);
+  if (e != cudaSuccess) return e;
+  if (unit == 2)
+    e = norm ? launch_t<kFmtNV, 2, true, false, kTensor>(p, st) : launch_t<kFmtNV, 2, false, false, kTensor>(p, st);
+  else
+    e = norm ? launch_t<kFmtNV, 1, true, false, kTensor>(p, st) : launch_t<kFmtNV, 1, false, false, kTensor>(p, st);
+  if (e != cudaSuccess) return e;
+  fill_row_scale<<<1, 1024, 0, st>>>(p.row_scale, p.T);
+  return cudaGetLastError();
 }
 
 }  // namespace sharq

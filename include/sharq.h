@@ -153,6 +153,17 @@ int sharq_prepare(const void *x_bf16_dev, int tokens, int k, const void *gamma_b
                   float eps, int nm_n, int nm_m, int unit, int fmt, sharq_prep *out,
                   void *stream);
 
+/* sharq_prepare with ONE NVFP4 second-level scale for the whole activation tensor instead
+ * of one per row: s_x = fp32(amax|xh|/2688) over every row (the stricter reading of NVFP4's
+ * "fp32 tensor scale"), shared by backbone and residual; row_scale receives that value in
+ * every entry, so sharq_linear consumes the result unchanged. Three launches (a tensor-amax
+ * pass over x, the preparation, a fill of row_scale) plus a 4-byte clear of row_scale[0],
+ * which holds the tensor amax in between. MXFP4 has no second-level scale: same as
+ * sharq_prepare. Arguments, layouts and errors as sharq_prepare. */
+int sharq_prepare_tensor_scale(const void *x_bf16_dev, int tokens, int k, const void *gamma_bf16_dev,
+                               float eps, int nm_n, int nm_m, int unit, int fmt, sharq_prep *out,
+                               void *stream);
+
 /* The preparation operator fed by a gate/up projection's output (one launch): the down
  * projection's input x = SiLU(g) * u is formed in registers from [g | u] and prepared as
  * by sharq_prepare without normalization, so x never goes through memory. The abstract's
