@@ -345,6 +345,11 @@ def run_sharq(args, rank, world, local):
     torch.cuda.synchronize()
     t_unf = graph_time(capture(unfused), n_gu)
     sw_bytes = T * Kd * (4 + PREP_BYTES_PER_ELEM - 2) + T * 4
+    # ---- one NVFP4 second-level scale per tensor (amax pass + preparation + scale fill)
+    p_ts = S.alloc_prep(T, K, 2, 4, 2, "nvfp4")
+    torch.cuda.synchronize()
+    t_ts = graph_time(capture(lambda st: [S.sharq_prepare_tensor_scale(xs[s], gamma, lin.eps, out=p_ts, stream=st)
+                                          for s in range(nsets)]), nsets)
     sw_gbs = sw_bytes / (t_sw / 1e3) / 1e9
     del gus
 
@@ -432,7 +437,11 @@ def run_sharq(args, rank, world, local):
         "next": {"swiglu_prep": {
             "workload": f"llama31_8b_down_from_gate_up T={T} K={Kd} nvfp4 2:4-pairs (x = SiLU(g)*u in the kernel)",
             "t_us": t_sw * 1e3, "achieved_gbs": sw_gbs, "bound": "hbm", "peak_gbs": hbm_peak,
-            "frac": sw_gbs / hbm_peak, "unfused_torch_swiglu_plus_prep_us": t_unf * 1e3}},
+            "frac": sw_gbs / hbm_peak, "unfused_torch_swiglu_plus_prep_us": t_unf * 1e3},
+            "tensor_scale_prep": {
+                "workload": f"llama31_8b_qkv_prefill T={T} K={K} nvfp4 2:4-pairs fused-rmsnorm, one scale per tensor",
+                "t_us": t_ts * 1e3, "per_row_scale_prep_us": t_prep_ms * 1e3,
+                "note": "3 launches + 4-byte clear; the amax pass reads x a second time"}},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "device_status": status,
