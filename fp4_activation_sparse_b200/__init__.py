@@ -14,6 +14,7 @@ Quantization for LLM Inference", Abstract):
   sharq_prepare_swiglu - the same operator on a down projection's gated input SiLU(g)*u
   sharq_prepare_tensor_scale - the same operator with one NVFP4 second-level scale per tensor
   sharq_linear       - sparse FP4 GEMM + dense FP4 GEMM into one output
+  sharq_linear_grouped - the same for many experts (mixture of experts) in one launch
 and the library's dense FP4 baseline (the README's "NVFP4" mode):
   sharq_quantize_dense, sharq_linear_dense.
 """
@@ -68,6 +69,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sharq_prepare_swiglu": (I, [P, I, I, I, I, I, I, ctypes.POINTER(_Prep), P]),
         "sharq_prepare_tensor_scale": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P]),
         "sharq_linear": (I, [ctypes.POINTER(_Prep), ctypes.POINTER(_WPack), P, I, P]),
+        "sharq_linear_grouped": (I, [ctypes.POINTER(_Prep), ctypes.POINTER(_WPack), ctypes.POINTER(P), I, I, P]),
         "sharq_quantize_dense": (I, [P, I, I, P, F, I, P, P, P]),
         "sharq_linear_dense": (I, [P, P, I, I, ctypes.POINTER(_WPack), P, I, P]),
         "sharq_device_status": (I, [P]),
@@ -260,6 +262,22 @@ def sharq_linear(prep: Prep, w: WPack, y: torch.Tensor | None = None, out_dtype=
     code = SHARQ_OUT_F32 if y.dtype == torch.float32 else SHARQ_OUT_BF16
     _check(lib.sharq_linear(ctypes.byref(prep.struct()), ctypes.byref(w.struct()), _ptr(y), code, _stream(stream)))
     return y
+
+
+def sharq_linear_grouped(preps: list[Prep], ws: list[WPack], ys: list[torch.Tensor] | None = None,
+                         out_dtype=torch.bfloat16, stream=None) -> list[torch.Tensor]:
+    """Mixture-of-experts form: Y_e = sharq_linear(preps[e], ws[e]) for every expert in one
+    launch (per 32 experts). Every weight shares n_out and k."""
+    n = len(preps)
+    assert n == len(ws) and n >= 1
+    if ys is None:
+        ys = [torch.empty(p.tokens, w.n_out, dtype=out_dtype, device=p.tiles.device) for p, w in zip(preps, ws)]
+    code = SHARQ_OUT_F32 if ys[0].dtype == torch.float32 else SHARQ_OUT_BF16
+    a = (_Prep * n)(*[p.struct() for p in preps])
+    w = (_WPack * n)(*[x.struct() for x in ws])
+    y = (ctypes.c_void_p * n)(*[t.data_ptr() for t in ys])
+    _check(lib.sharq_linear_grouped(a, w, y, n, code, _stream(stream)))
+    return ys
 
 
 @dataclass

@@ -218,7 +218,8 @@ static int run_gemm(sharq::GemmParams &g, const char *name, cudaStream_t st) {
   return SHARQ_OK;
 }
 
-int sharq_linear(const sharq_prep *a, const sharq_wpack *w, void *y, int out_dtype, void *stream) {
+// Checks one (prep, weight, output) problem of sharq_linear / sharq_linear_grouped.
+static int check_linear(const sharq_prep *a, const sharq_wpack *w, const void *y, int out_dtype) {
   if (!a || !y) return fail(SHARQ_ERR_INVALID_ARG, "null prep or output");
   if (int s = check_wpack(w)) return s;
   if (!valid_fmt(a->fmt)) return fail(SHARQ_ERR_INVALID_ARG, "prep has unknown fmt %d", a->fmt);
@@ -233,22 +234,64 @@ int sharq_linear(const sharq_prep *a, const sharq_wpack *w, void *y, int out_dty
   if (!a->tiles || !a->row_scale) return fail(SHARQ_ERR_INVALID_ARG, "null buffer in prep");
   if (!aligned16(a->tiles) || !aligned16(a->row_scale) || !aligned16(y))
     return fail(SHARQ_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
+  return 0;
+}
+
+static void set_group(sharq::GemmGroup &G, const void *tiles, const float *row_scale, int tokens,
+                      const sharq_wpack *w, void *y) {
+  G.a_tiles = static_cast<const uint8_t *>(tiles);
+  G.row_scale = row_scale;
+  G.w_tiles = static_cast<const uint8_t *>(w->tiles);
+  G.tensor_scale = w->tensor_scale;
+  G.y = y;
+  G.T = tokens;
+  G.T_pad = sharq::round_up(tokens, 256);
+}
+
+int sharq_linear(const sharq_prep *a, const sharq_wpack *w, void *y, int out_dtype, void *stream) {
+  if (int s = check_linear(a, w, y, out_dtype)) return s;
   sharq::GemmParams g;
   memset(&g, 0, sizeof g);
-  g.a_tiles = static_cast<const uint8_t *>(a->tiles);
-  g.row_scale = a->row_scale;
-  g.w_tiles = static_cast<const uint8_t *>(w->tiles);
-  g.tensor_scale = w->tensor_scale;
-  g.y = y;
-  g.T = a->tokens;
+  set_group(g.grp[0], a->tiles, a->row_scale, a->tokens, w, y);
+  g.n_groups = 1;
   g.N = w->n_out;
   g.K = a->k;
-  g.T_pad = sharq::round_up(a->tokens, 256);
   g.N_pad = sharq::round_up(w->n_out, 256);
   g.fmt = a->fmt;
   g.out_f32 = out_dtype == SHARQ_OUT_F32;
   g.sparse = 1;
   return run_gemm(g, "sharq_linear", static_cast<cudaStream_t>(stream));
+}
+
+int sharq_linear_grouped(const sharq_prep *a, const sharq_wpack *w, void *const *y, int n_groups, int out_dtype,
+                         void *stream) {
+  if (!a || !w || !y) return fail(SHARQ_ERR_INVALID_ARG, "null group arrays");
+  if (n_groups < 1) return fail(SHARQ_ERR_INVALID_ARG, "n_groups must be >= 1 (got %d)", n_groups);
+  for (int e = 0; e < n_groups; ++e) {
+    if (a[e].tokens == 0 && y[e]) continue;  // an expert without tokens: nothing to do
+    if (int s = check_linear(&a[e], &w[e], y[e], out_dtype)) return s;
+    if (w[e].n_out != w[0].n_out || w[e].k != w[0].k || w[e].fmt != w[0].fmt)
+      return fail(SHARQ_ERR_INVALID_ARG, "group %d: every weight must have the shape and format of group 0", e);
+  }
+  if (int s = check_wpack(&w[0])) return s;
+  for (int e0 = 0; e0 < n_groups; e0 += sharq::kMaxGroups) {  // one launch per kMaxGroups groups
+    sharq::GemmParams g;
+    memset(&g, 0, sizeof g);
+    const int n = n_groups - e0 < sharq::kMaxGroups ? n_groups - e0 : sharq::kMaxGroups;
+    for (int i = 0; i < n; ++i) {
+      const sharq_prep &ae = a[e0 + i];
+      set_group(g.grp[i], ae.tiles, ae.row_scale, ae.tokens > 0 ? ae.tokens : 0, &w[e0 + i], y[e0 + i]);
+    }
+    g.n_groups = n;
+    g.N = w[0].n_out;
+    g.K = w[0].k;
+    g.N_pad = sharq::round_up(w[0].n_out, 256);
+    g.fmt = w[0].fmt;
+    g.out_f32 = out_dtype == SHARQ_OUT_F32;
+    g.sparse = 1;
+    if (int s = run_gemm(g, "sharq_linear_grouped", static_cast<cudaStream_t>(stream))) return s;
+  }
+  return SHARQ_OK;
 }
 
 int sharq_linear_dense(const void *tiles, const float *row_scale, int tokens, int k, const sharq_wpack *w, void *y,
@@ -262,15 +305,10 @@ int sharq_linear_dense(const void *tiles, const float *row_scale, int tokens, in
     return fail(SHARQ_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
   sharq::GemmParams g;
   memset(&g, 0, sizeof g);
-  g.a_tiles = static_cast<const uint8_t *>(tiles);
-  g.row_scale = row_scale;
-  g.w_tiles = static_cast<const uint8_t *>(w->tiles);
-  g.tensor_scale = w->tensor_scale;
-  g.y = y;
-  g.T = tokens;
+  set_group(g.grp[0], tiles, row_scale, tokens, w, y);
+  g.n_groups = 1;
   g.N = w->n_out;
   g.K = k;
-  g.T_pad = sharq::round_up(tokens, 256);
   g.N_pad = sharq::round_up(w->n_out, 256);
   g.fmt = w->fmt;
   g.out_f32 = out_dtype == SHARQ_OUT_F32;

@@ -320,9 +320,24 @@ __device__ __forceinline__ void reg_fence32(uint32_t *r) {
                  "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 }
 
-template <bool MX, bool SPARSE>
+// Group of a pair tile (groups hold consecutive tile ranges; empty groups are skipped).
+template <int MAXG>
+__device__ __forceinline__ int group_of(const GemmParams &p, int tile) {
+  int g = 0;
+  if (MAXG > 1)
+    while (g + 1 < p.n_groups && tile >= p.grp[g + 1].tile_begin) ++g;
+  return g;
+}
+
+template <int MAXG>
+struct __align__(64) TmaMapSet {
+  TmaMaps m[MAXG];
+};
+
+// MAXG: 1 for one problem per launch, kMaxGroups for the grouped (mixture-of-experts) form.
+template <bool MX, bool SPARSE, int MAXG>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    sharq_gemm_kernel(const __grid_constant__ TmaMaps maps, GemmParams p) {
+    sharq_gemm_kernel(const __grid_constant__ TmaMapSet<MAXG> ms, const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOutOffset + kEpiWarps * kStageOutBytes);
@@ -346,8 +361,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   using L = Stage<MX, SPARSE>;
   constexpr int apt_res = atoms_res(MX ? 1 : 0), apt_sp = atoms_sp(MX ? 1 : 0);
   constexpr int kStageBytes = L::kBytes;
-  const int num_m = (p.T + 2 * BM - 1) / (2 * BM), num_n = (p.N + BN - 1) / BN, num_k = p.K / BK;
-  const int num_tiles = num_m * num_n;
+  const int num_k = p.K / BK;
+  const int num_tiles = p.num_tiles;
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
   const uint64_t limit = p.wait_limit > 0 ? (uint64_t)p.wait_limit : 4000000000ull;
 
@@ -366,8 +381,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0 && lane == 0) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.act) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.w) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&ms.m[0].act) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&ms.m[0].w) : "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -388,8 +403,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool issued = false, ok = true;
       const uint32_t full_leader0 = map_to_rank(full_bar(0), 0);
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int m0 = (tile % num_m) * (2 * BM) + (int)rank * BM;  // this CTA's activation rows
-        const int n0 = (tile / num_m) * BN;                          // the pair's output columns
+        const int g = group_of<MAXG>(p, tile), lt = tile - p.grp[g].tile_begin, num_m = p.grp[g].num_m;
+        const TmaMaps &maps = ms.m[g];
+        const int m0 = (lt % num_m) * (2 * BM) + (int)rank * BM;  // this CTA's activation rows
+        const int n0 = (lt / num_m) * BN;                          // the pair's output columns
         const int a_row0 = (m0 / 128) * num_k * (L::A.bytes / 1024);  // chunk rows of 1024 bytes
         const int w_row0 = (n0 / 128 + (int)rank) * num_k * (L::W.bytes / 1024);
         for (int kt = 0; kt < num_k; ++kt) {
@@ -489,16 +506,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t acc_empty_leader = map_to_rank(acc_empty, 0);
     const uint32_t out_smem = smem0 + kOutOffset + (warp - 2) * kStageOutBytes;
     uint32_t acc_phase = 0;
-    const float s_w = p.tensor_scale[0];
     for (int tile = pair; tile < num_tiles; tile += num_pairs) {
-      const int m0 = (tile % num_m) * (2 * BM) + (int)rank * BM, n0 = (tile / num_m) * BN;
+      const int g = group_of<MAXG>(p, tile), lt = tile - p.grp[g].tile_begin, num_m = p.grp[g].num_m;
+      const GemmGroup &G = p.grp[g];
+      const float s_w = G.tensor_scale[0];
+      const int m0 = (lt % num_m) * (2 * BM) + (int)rank * BM, n0 = (lt / num_m) * BN;
       const int row = m0 + r_local;
-      const float scale = row < p.T ? __fmul_rn(p.row_scale[row], s_w) : 0.f;
+      const float scale = row < G.T ? __fmul_rn(G.row_scale[row], s_w) : 0.f;
       if (!mbar_wait(acc_full, acc_phase, limit, abort_flag)) break;
       tc_fence_after();
       const uint32_t tacc = tmem + ((uint32_t)(quarter * 32) << 16) + col_half * 128;
       const int col0 = n0 + col_half * 128;
-      const bool row_ok = row < p.T;
+      const bool row_ok = row < G.T;
       if (p.out_f32) {
         // float32 output: 32 columns at a time, the tensor memory held until the last load
 #pragma unroll 1
@@ -509,7 +528,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           reg_fence32(r);
           const int col = col0 + 32 * c;
           if (!row_ok || col >= p.N) continue;
-          float *dst = reinterpret_cast<float *>(p.y) + (size_t)row * p.N + col;
+          float *dst = reinterpret_cast<float *>(G.y) + (size_t)row * p.N + col;
           if (col + 32 <= p.N) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
@@ -568,7 +587,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           fence_proxy_async();
           __syncwarp();
           if (lane == 0) {
-            if (row0 < p.T && col0 + 32 * c < p.N) tma_store_2d(&maps.y, out_smem, col0 + 32 * c, row0);
+            if (row0 < G.T && col0 + 32 * c < p.N) tma_store_2d(&ms.m[g].y, out_smem, col0 + 32 * c, row0);
             bulk_commit();
           }
         }
@@ -707,8 +726,8 @@ struct MapCache {
 
 constexpr int kMaxDevices = 64;
 
-template <bool MX, bool SPARSE>
-cudaError_t launch_t(const TmaMaps &maps, const GemmParams &p, cudaStream_t st) {
+template <bool MX, bool SPARSE, int MAXG>
+cudaError_t launch_t(const TmaMapSet<MAXG> &ms, const GemmParams &p, cudaStream_t st) {
   static std::once_flag once[kMaxDevices];
   static cudaError_t setup_err[kMaxDevices];
   static int sms[kMaxDevices];
@@ -717,50 +736,73 @@ cudaError_t launch_t(const TmaMaps &maps, const GemmParams &p, cudaStream_t st) 
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::call_once(once[dev], [dev] {
-    setup_err[dev] = cudaFuncSetAttribute(sharq_gemm_kernel<MX, SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          kSmemBytes);
+    setup_err[dev] = cudaFuncSetAttribute(sharq_gemm_kernel<MX, SPARSE, MAXG>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (setup_err[dev] == cudaSuccess)
       setup_err[dev] = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
   });
   if (setup_err[dev] != cudaSuccess) return setup_err[dev];
-  const int tiles = ((p.T + 2 * BM - 1) / (2 * BM)) * ((p.N + BN - 1) / BN);
-  const int pairs = tiles < sms[dev] / 2 ? tiles : sms[dev] / 2;
-  sharq_gemm_kernel<MX, SPARSE><<<2 * pairs, kThreads, kSmemBytes, st>>>(maps, p);
+  if (p.num_tiles == 0) return cudaSuccess;
+  const int pairs = p.num_tiles < sms[dev] / 2 ? p.num_tiles : sms[dev] / 2;
+  sharq_gemm_kernel<MX, SPARSE, MAXG><<<2 * pairs, kThreads, kSmemBytes, st>>>(ms, p);
   return cudaGetLastError();
 }
 
-}  // namespace
-
-cudaError_t launch_gemm(const GemmParams &p, cudaStream_t st, const char **why) {
+// Tensor maps of one group: activation and weight chunks (cached), bf16 output.
+bool group_maps(TmaMaps *maps, const GemmParams &p, const GemmGroup &G) {
   static MapCache cache;
-  TmaMaps maps;
   const int fmt = p.fmt == kFmtMX ? 1 : 0;
   const ActTile A = act_tile(fmt, 2, p.sparse != 0);
   const WTile W = w_tile(fmt);
   const uint64_t ks = (uint64_t)p.K / BK;
-  const uint64_t a_rows = (uint64_t)(p.T_pad / 128) * ks * (A.bytes / 1024);
+  const uint64_t a_rows = (uint64_t)(G.T_pad / 128) * ks * (A.bytes / 1024);
   const uint64_t w_rows = (uint64_t)(p.N_pad / 128) * ks * (W.bytes / 1024);
-  bool y_ok = true;
-  if (!p.out_f32) {
+  memset(&maps->y, 0, sizeof maps->y);
+  if (!p.out_f32 && G.T > 0) {
     auto fn = encode_fn();
-    cuuint64_t dims[2] = {(cuuint64_t)p.N, (cuuint64_t)p.T};
+    cuuint64_t dims[2] = {(cuuint64_t)p.N, (cuuint64_t)G.T};
     cuuint64_t strides[1] = {(cuuint64_t)p.N * 2};
     cuuint32_t box[2] = {32, 32};
     cuuint32_t estr[2] = {1, 1};
-    y_ok = fn && fn(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.y, dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-  } else {
-    memset(&maps.y, 0, sizeof maps.y);
+    if (!fn || fn(&maps->y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, G.y, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
   }
-  if (!y_ok || !cache.get(&maps.act, p.a_tiles, a_rows, A.bytes / 1024) ||
-      !cache.get(&maps.w, p.w_tiles, w_rows, W.bytes / 1024)) {
-    *why = "cuTensorMapEncodeTiled failed (driver entry point missing or operand layout rejected)";
-    return cudaErrorInvalidValue;
+  if (G.T == 0) {  // no tiles: the maps are never used
+    memset(&maps->act, 0, sizeof maps->act);
+    memset(&maps->w, 0, sizeof maps->w);
+    return true;
   }
+  return cache.get(&maps->act, G.a_tiles, a_rows, A.bytes / 1024) && cache.get(&maps->w, G.w_tiles, w_rows, W.bytes / 1024);
+}
+
+template <int MAXG>
+cudaError_t launch_groups(const GemmParams &p, cudaStream_t st, const char **why) {
+  TmaMapSet<MAXG> ms;
+  for (int g = 0; g < p.n_groups; ++g)
+    if (!group_maps(&ms.m[g], p, p.grp[g])) {
+      *why = "cuTensorMapEncodeTiled failed (driver entry point missing or operand layout rejected)";
+      return cudaErrorInvalidValue;
+    }
   const bool mx = p.fmt == kFmtMX;
-  if (p.sparse) return mx ? launch_t<true, true>(maps, p, st) : launch_t<false, true>(maps, p, st);
-  return mx ? launch_t<true, false>(maps, p, st) : launch_t<false, false>(maps, p, st);
+  if (p.sparse) return mx ? launch_t<true, true, MAXG>(ms, p, st) : launch_t<false, true, MAXG>(ms, p, st);
+  return mx ? launch_t<true, false, MAXG>(ms, p, st) : launch_t<false, false, MAXG>(ms, p, st);
+}
+
+}  // namespace
+
+// Fills the tile ranges of p.grp[0 .. n_groups) and launches one kernel.
+cudaError_t launch_gemm(GemmParams p, cudaStream_t st, const char **why) {
+  int tiles = 0;
+  const int num_n = (p.N + BN - 1) / BN;
+  for (int g = 0; g < p.n_groups; ++g) {
+    p.grp[g].num_m = (p.grp[g].T + 2 * BM - 1) / (2 * BM);
+    p.grp[g].tile_begin = tiles;
+    tiles += p.grp[g].num_m * num_n;
+  }
+  p.num_tiles = tiles;
+  return p.n_groups == 1 ? launch_groups<1>(p, st, why) : launch_groups<kMaxGroups>(p, st, why);
 }
 
 cudaError_t read_and_clear_device_status(int *status, cudaStream_t st) {

@@ -63,13 +63,23 @@ struct PackParams {
   float *tensor_scale;  // [0] s_w, [1] amax
 };
 
-struct GemmParams {
+// One GEMM problem of a (possibly grouped) launch: Y_g = A_g . W_g^T.
+struct GemmGroup {
   const uint8_t *a_tiles;     // activation chunks: SharQ prep (sparse) or dense quantizer
   const float *row_scale;     // [T]
   const uint8_t *w_tiles;     // weight chunks
   const float *tensor_scale;  // [0] = s_w
   void *y;                    // [T][N]
-  int T, N, K, T_pad, N_pad;
+  int T, T_pad;
+  int tile_begin, num_m;      // first pair tile of this group in the launch, its 256-row blocks
+};
+
+constexpr int kMaxGroups = 32;  // groups per launch of the grouped GEMM
+
+struct GemmParams {
+  GemmGroup grp[kMaxGroups];
+  int n_groups, num_tiles;    // num_tiles: pair tiles over all groups
+  int N, K, N_pad;            // shared by every group
   int fmt, out_f32, sparse;
   long long wait_limit;
 };
@@ -77,7 +87,7 @@ struct GemmParams {
 cudaError_t launch_prep(PrepParams p, int fmt, int unit, bool norm, bool dense, bool swiglu, cudaStream_t st);
 cudaError_t launch_prep_tensor_scale(PrepParams p, int unit, bool norm, cudaStream_t st);
 cudaError_t launch_pack(PackParams p, int fmt, cudaStream_t st);
-cudaError_t launch_gemm(const GemmParams &p, cudaStream_t st, const char **why);
+cudaError_t launch_gemm(GemmParams p, cudaStream_t st, const char **why);
 cudaError_t read_and_clear_device_status(int *status, cudaStream_t st);
 
 }  // namespace sharq

@@ -188,6 +188,18 @@ int sharq_prepare_swiglu(const void *gate_up_bf16_dev, int tokens, int k, int nm
 int sharq_linear(const sharq_prep *a, const sharq_wpack *w, void *y_dev, int out_dtype,
                  void *stream);
 
+/* Grouped (mixture-of-experts) SharQ linear: n_groups independent problems
+ * Y_e = sharq_linear(a[e], w[e]) computed by one launch per 32 groups, the CTA pairs working
+ * through the output tiles of all groups (each expert's tokens prepared by sharq_prepare into
+ * their own buffers, so no tile mixes experts). The abstract evaluates a mixture-of-experts
+ * model (Qwen3-30B-A3B) with the method; this is its expert layer.
+ *   a[e], w[e]  prepared activation and packed weight of group e; every weight has the same
+ *               n_out, k and fmt; a[e].tokens == 0 marks an expert without tokens (skipped)
+ *   y_dev[e]    [a[e].tokens][n_out] output of group e (bf16 or float32 per out_dtype)
+ * Checks and errors as sharq_linear, per group. */
+int sharq_linear_grouped(const sharq_prep *a, const sharq_wpack *w, void *const *y_dev, int n_groups,
+                         int out_dtype, void *stream);
+
 /* The library's own dense FP4 baseline (the README's "NVFP4: dense FP4 baseline"):
  * optional RMSNorm + dense block quantization of xh with the same row-scale rule
  * (one launch), and a dense FP4 GEMM against the weight's dense view (one launch).
