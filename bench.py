@@ -345,6 +345,47 @@ def run_sharq(args, rank, world, local):
     torch.cuda.synchronize()
     t_unf = graph_time(capture(unfused), n_gu)
     sw_bytes = T * Kd * (4 + PREP_BYTES_PER_ELEM - 2) + T * 4
+    # ---- mixture of experts: Qwen3-30B-A3B expert gate/up projections (K=2048, N=2*768) for
+    # T tokens routed top-8 of 128. The routed rows are laid out expert by expert, each
+    # expert's group padded to 256 rows, prepared by ONE sharq_prepare over all of them, and
+    # every expert's view of that buffer goes to one grouped GEMM launch.
+    moe = wl.QWEN3_MOE
+    Km, Nm, E = moe["hidden"], 2 * moe["moe_intermediate"], moe["n_experts"]
+    route = wl.moe_routing(replica_seed(rank), T, E, moe["top_k"])
+    counts = np.bincount(route.reshape(-1), minlength=E)
+    starts = np.concatenate([[0], np.cumsum((counts + 255) // 256 * 256)])[:-1]
+    rows_pad = int(starts[-1] + (counts[-1] + 255) // 256 * 256)
+    order = np.argsort(route.reshape(-1), kind="stable")            # assignments sorted by expert
+    src_tok = (order // moe["top_k"]).astype(np.int64)
+    dst_row = np.concatenate([starts[e] + np.arange(counts[e]) for e in range(E)]).astype(np.int64)
+    x_moe_tok = to_dev(wl.outlier_activations(np.random.default_rng(replica_seed(rank) + 600), T, Km,
+                                              max(2, Km // 100), 20.0, 100.0, 0.5))
+    x_moe = torch.zeros(rows_pad, Km, dtype=torch.bfloat16, device="cuda")
+    x_moe[torch.from_numpy(dst_row).cuda()] = x_moe_tok[torch.from_numpy(src_tok).cuda()]
+    gen = torch.Generator(device="cuda").manual_seed(1234 + rank)
+    wps_moe = []
+    for e in range(E):
+        w_e = (torch.randn(Nm, Km, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)
+        wps_moe.append(S.sharq_pack_weight(w_e, "nvfp4"))
+    del w_e
+    p_moe = S.alloc_prep(rows_pad, Km, 2, 4, 2, "nvfp4")
+    chunk = p_moe.tiles.numel() // (rows_pad // 128)               # bytes per 128-row block
+    views = [S.Prep(p_moe.tiles[int(starts[e]) // 128 * chunk:], p_moe.row_scale[int(starts[e]):],
+                    int(counts[e]), Km, 2, 4, 2, S.SHARQ_NVFP4) for e in range(E)]
+    ys_moe = [torch.empty(max(int(c), 1), Nm, dtype=torch.bfloat16, device="cuda") for c in counts]
+    S.sharq_prepare(x_moe, None, 1e-6, out=p_moe)
+    S.sharq_linear_grouped(views, wps_moe, ys_moe)
+    torch.cuda.synchronize()
+    t_moe_prep = graph_time(capture(lambda st: S.sharq_prepare(x_moe, None, 1e-6, out=p_moe, stream=st)), 1)
+    t_moe_gemm = graph_time(capture(lambda st: S.sharq_linear_grouped(views, wps_moe, ys_moe, stream=st)), 1)
+    moe_work = 3.0 * int(counts.sum()) * Nm * Km                     # dense-equivalent, routed rows only
+    moe_tflops = moe_work / (t_moe_gemm / 1e3) / 1e12
+    moe_line = {"workload": f"qwen3_30b_a3b experts gate_up T={T} top-{moe['top_k']} of {E}, K={Km} N={Nm} nvfp4",
+                "routed_rows": int(counts.sum()), "padded_rows": rows_pad, "launches": "1 prep + "
+                f"{(E + 31) // 32} grouped GEMM", "t_prep_us": t_moe_prep * 1e3, "t_grouped_gemm_us": t_moe_gemm * 1e3,
+                "achieved_tflops": moe_tflops, "peak_tflops": fp4_dense_peak, "frac": moe_tflops / fp4_dense_peak}
+    del x_moe, x_moe_tok, wps_moe, p_moe, views, ys_moe
+
     # ---- one NVFP4 second-level scale per tensor (amax pass + preparation + scale fill)
     p_ts = S.alloc_prep(T, K, 2, 4, 2, "nvfp4")
     torch.cuda.synchronize()
@@ -441,7 +482,8 @@ def run_sharq(args, rank, world, local):
             "tensor_scale_prep": {
                 "workload": f"llama31_8b_qkv_prefill T={T} K={K} nvfp4 2:4-pairs fused-rmsnorm, one scale per tensor",
                 "t_us": t_ts * 1e3, "per_row_scale_prep_us": t_prep_ms * 1e3,
-                "note": "3 launches + 4-byte clear; the amax pass reads x a second time"}},
+                "note": "3 launches + 4-byte clear; the amax pass reads x a second time"},
+            "moe_grouped": moe_line},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "device_status": status,

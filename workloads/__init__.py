@@ -156,6 +156,17 @@ def dit(seed: int = 4, T: int = 32760) -> Linear:
     return Linear(f"dit_{T}x{K}x{N}", x, None, weight(rng, N, K))
 
 
+def moe_routing(seed: int, T: int, n_experts: int, top_k: int) -> np.ndarray:
+    """Expert ids [T, top_k] of a mixture-of-experts router: the top_k of seeded N(0, 1)
+    logits per token (distinct experts, token-major)."""
+    rng = np.random.default_rng(seed + 500)
+    logits = rng.standard_normal((T, n_experts), dtype=np.float32)
+    return np.argsort(-logits, axis=1, kind="stable")[:, :top_k].astype(np.int64)
+
+
+QWEN3_MOE = dict(hidden=2048, moe_intermediate=768, n_experts=128, top_k=8)  # Qwen3-30B-A3B expert layer
+
+
 def crafted_row(values) -> np.ndarray:
     """bf16 bits of a hand-written row (for edge-case tests)."""
     return f32_to_bf16_bits(np.asarray(values, dtype=np.float32)[None, :])
