@@ -393,6 +393,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync();  // barriers initialized and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Launched as a programmatic dependent of the preparation: the prologue above overlaps its
+  // tail; its outputs are read only after it has completed and flushed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -744,7 +747,18 @@ cudaError_t launch_t(const TmaMapSet<MAXG> &ms, const GemmParams &p, cudaStream_
   if (setup_err[dev] != cudaSuccess) return setup_err[dev];
   if (p.num_tiles == 0) return cudaSuccess;
   const int pairs = p.num_tiles < sms[dev] / 2 ? p.num_tiles : sms[dev] / 2;
-  sharq_gemm_kernel<MX, SPARSE, MAXG><<<2 * pairs, kThreads, kSmemBytes, st>>>(ms, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may start while the previous kernel drains
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, sharq_gemm_kernel<MX, SPARSE, MAXG>, ms, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

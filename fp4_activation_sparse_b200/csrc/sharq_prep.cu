@@ -432,6 +432,9 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   const int stride = 32 * W;
   const bool live_row = row < p.T;
 
+  // A GEMM launched after this kernel as its programmatic dependent may start its prologue on
+  // SMs this grid leaves; it reads our outputs only after this grid has completed.
+  asm volatile("griddepcontrol.launch_dependents;");
   uint32_t xr[kMaxDP][8];
 #pragma unroll
   for (int i = 0; i < kMaxDP; ++i) {
