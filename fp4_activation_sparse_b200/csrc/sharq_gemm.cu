@@ -120,13 +120,16 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
-// arrive on a barrier given by its shared::cluster address (own or peer CTA)
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+// Arrive on a barrier given by its shared::cluster address (own or peer CTA), relaxed (no
+// release ordering of this thread's memory operations): for handing back
+// tensor memory whose loads have completed (tcgen05.wait::ld) -- nothing in memory is handed
+// over, and a cluster-scope release was measured to stall the arriving thread ~1400 cycles.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-// CLUSTER: acquire at cluster scope, pairing with the peer CTA's release-arrive; otherwise
-// CTA scope (barriers completed by TMA transactions or tcgen05.commit).
+// CLUSTER: acquire at cluster scope (the accumulator hand-back, arrived on from both CTAs);
+// otherwise CTA scope (barriers completed by TMA transactions or tcgen05.commit).
 template <bool CLUSTER>
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -546,7 +549,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+        if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_leader);
       } else {
         // bf16 output: this warp's 32 rows x 128 columns are read and rounded first (64
         // registers of packed pairs), the tensor memory is handed back, and the stores
@@ -571,7 +574,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+        if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_leader);
         // Write this warp's 32 x 128 block with bulk tensor stores (coalesced; rows >= T and
         // columns >= N clipped by the tensor map) through a 2 KB staging box of 32 x 32, in
         // 64-byte-swizzled rows: 16-byte unit u of row r at u ^ ((r / 2) % 4), conflict-free.
