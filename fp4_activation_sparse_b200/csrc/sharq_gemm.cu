@@ -567,8 +567,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const __nv_bfloat162 v = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[c][2 * i]), scale),
-                                                             __fmul_rn(__uint_as_float(r[c][2 * i + 1]), scale));
+              // packed product (round to nearest per lane; it feeds only the bf16 conversion)
+              float y0 = __uint_as_float(r[c][2 * i]), y1 = __uint_as_float(r[c][2 * i + 1]);
+              asm("{\n\t.reg .b64 x, s, z;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 s, {%2, %2};\n\t"
+                  "mul.rn.f32x2 z, x, s;\n\tmov.b64 {%0, %1}, z;\n\t}"
+                  : "+f"(y0), "+f"(y1)
+                  : "f"(scale));
+              const __nv_bfloat162 v = __floats2bfloat162_rn(y0, y1);
               packed[2 * h + c][i] = *reinterpret_cast<const uint32_t *>(&v);
             }
         }
