@@ -23,18 +23,22 @@
 //               Both paths carry the same per-row scale s_x, so one accumulator holds their
 //               sum. Each weight chunk feeds both MMAs. Commits arrive on both CTAs'
 //               barriers (multicast commit).
-//   warps 10-14 scale copiers (leader): tcgen05.cp of the K step's scales and metadata into one
-//               of three tensor-memory buffers, split five ways (dense-view weight scales of
-//               the first and second K halves, sparse-view weight scales, residual scales,
-//               backbone scales + metadata), each from its own thread: a copy costs its
-//               issuing thread tens of cycles, so the copies keep pace with the MMAs only
-//               when spread over several threads.
 //   warps 2..9  epilogue (both CTAs): tcgen05.ld of the accumulator, y = acc * s_x[row] * s_w
 //               rounded to bf16 in registers, the tensor memory handed back, then the block
 //               staged in shared memory and written by bulk tensor stores (coalesced, clipped at
 //               the tensor's edges) while the next tile's MMAs run. Row-wise 16-byte stores
 //               from registers took a quarter of the kernel's time and delayed the next tile's
 //               loads. (float32 output, a test format, is stored from registers.)
+//   warps 10-14 scale copiers (leader): tcgen05.cp of the K step's scales and metadata into one
+//               of three tensor-memory buffers, split five ways (dense-view weight scales of
+//               the first and second K halves, sparse-view weight scales, residual scales,
+//               backbone scales + metadata), each from its own thread: a copy costs its
+//               issuing thread tens of cycles, so the copies keep pace with the MMAs only
+//               when spread over several threads.
+// One launch may cover several problems of the same N and K (the experts of a mixture-of-
+// experts layer): the persistent loop decodes each pair tile into (group, m-block, n-block)
+// from a prefix table of tile counts. The kernel is launched as a programmatic dependent of
+// the preparation and waits for it (griddepcontrol.wait) only after its prologue.
 // Every mbarrier wait is bounded by a time limit; on expiry the CTA records a status word,
 // stops issuing, drains (bounded) what it issued, frees TMEM and exits.
 #include <cuda.h>
