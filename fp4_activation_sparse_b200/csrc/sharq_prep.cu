@@ -36,7 +36,7 @@ namespace sharq {
 namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
-constexpr int kMaxDP = 8;  // double pieces (16 elements) per lane
+constexpr int kMaxDP = 8;  // double pieces (16 elements) per lane, at most
 
 // The two largest of four keys, ties to the lower index, as a metadata nibble i0 | i1 << 2
 // (i0 < i1); also returns the largest key. Tournament: winners and losers of (0,1) and
@@ -418,7 +418,7 @@ __device__ __forceinline__ void row_scales(int fmt, float amax, float &s_x, floa
 // written afterwards by fill_row_scale (blocks still read row_scale[0] while others finish).
 constexpr int kRow = 0, kSwiglu = 1, kAmax = 2, kTensor = 3;
 
-template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE>
+template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE, int DP>
 __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   extern __shared__ float4 gamma_smem4[];  // NORM: the RMSNorm weight as float32 (K rounded up to 512)
   __shared__ double sm_d[64];
@@ -435,9 +435,9 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   // A GEMM launched after this kernel as its programmatic dependent may start its prologue on
   // SMs this grid leaves; it reads our outputs only after this grid has completed.
   asm volatile("griddepcontrol.launch_dependents;");
-  uint32_t xr[kMaxDP][8];
+  uint32_t xr[DP][8];
 #pragma unroll
-  for (int i = 0; i < kMaxDP; ++i) {
+  for (int i = 0; i < DP; ++i) {
     const int dp = i * stride + wt * 32 + lane;
     if (live_row && dp < ndp_row) {
       const uint16_t *src = p.x + (size_t)row * p.x_stride + (size_t)dp * 16;
@@ -460,7 +460,7 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
     }
     double ss = 0.0;
 #pragma unroll
-    for (int i = 0; i < kMaxDP; ++i) {
+    for (int i = 0; i < DP; ++i) {
       const int dp = i * stride + wt * 32 + lane;
       if (live_row && dp < ndp_row) {
         // float64: bf16 squares are exact and the sum keeps ~2^-53 relative accuracy, so
@@ -479,7 +479,7 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
 
   float am = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxDP; ++i) {
+  for (int i = 0; i < DP; ++i) {
     const int dp = i * stride + wt * 32 + lane;
     if (live_row && dp < ndp_row) {
       float v[16];
@@ -505,7 +505,7 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   const size_t chunk_step = (size_t)2 * W * kChunk;
   const bool pad_row = !live_row && row < p.T_pad;
 #pragma unroll
-  for (int i = 0; i < kMaxDP; ++i) {
+  for (int i = 0; i < DP; ++i) {
     const int base = i * stride + wt * 32;  // warp-uniform
     if (base >= ndp_row) break;
     const int dp = base + lane;
@@ -541,8 +541,8 @@ __global__ void __launch_bounds__(1024) fill_row_scale(float *row_scale, int T) 
   for (int i = threadIdx.x; i < T; i += blockDim.x) row_scale[i] = s_x;
 }
 
-template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE = kRow>
-cudaError_t launch_t(const PrepParams &p, cudaStream_t st) {
+template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE, int DP>
+cudaError_t launch_k(const PrepParams &p, cudaStream_t st) {
   const int W = p.TS;
   const int teams = W >= 8 ? 1 : 8 / W;
   const int block = teams * W * 32;
@@ -558,13 +558,21 @@ cudaError_t launch_t(const PrepParams &p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [dev] {
-      err[dev] = cudaFuncSetAttribute(prep_kernel<FMT, UNIT, NORM, DENSE, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      err[dev] = cudaFuncSetAttribute(prep_kernel<FMT, UNIT, NORM, DENSE, MODE, DP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       32768 * (int)sizeof(float));
     });
     if (err[dev] != cudaSuccess) return err[dev];
   }
-  prep_kernel<FMT, UNIT, NORM, DENSE, MODE><<<grid, block, smem, st>>>(p);
+  prep_kernel<FMT, UNIT, NORM, DENSE, MODE, DP><<<grid, block, smem, st>>>(p);
   return cudaGetLastError();
+}
+
+// A single-warp row of at most 2048 elements needs 4 pieces per lane: the smaller register
+// array leaves room for more resident warps.
+template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE = kRow>
+cudaError_t launch_t(const PrepParams &p, cudaStream_t st) {
+  if (p.TS == 1 && p.K / 16 <= 32 * 4) return launch_k<FMT, UNIT, NORM, DENSE, MODE, 4>(p, st);
+  return launch_k<FMT, UNIT, NORM, DENSE, MODE, kMaxDP>(p, st);
 }
 
 template <int FMT, int UNIT, bool DENSE>
