@@ -267,6 +267,15 @@ def run_sharq(args, rank, world, local):
         return g
 
     step_graphs = [capture(lambda st, s=s: step(s, st)) for s in range(nsets)]
+    # one graph over all input sets' steps: consecutive steps then follow each other without
+    # a graph launch between them, as layers do inside a captured forward pass
+    run_graph = capture(lambda st: [step(s, st) for s in range(nsets)])
+
+    def run_steps(n):
+        for _ in range(n // nsets):
+            run_graph.replay()
+        for i in range(n % nsets):
+            step_graphs[i].replay()
     prep_graph = capture(lambda st: [S.sharq_prepare(xs[s], gamma, lin.eps, 2, 4, 2, "nvfp4", out=preps[s], stream=st)
                                      for s in range(nsets)])
     lin_graph = capture(lambda st: [S.sharq_linear(preps[s], wps[s], y=ys[s], stream=st) for s in range(nsets)])
@@ -279,15 +288,14 @@ def run_sharq(args, rank, world, local):
         t_end = time.perf_counter() + 1.0
         i = 0
         while time.perf_counter() < t_end:
-            step_graphs[i % nsets].replay()
+            run_graph.replay()
             i += 1
-            if i % 64 == 0:
+            if i % 8 == 0:
                 torch.cuda.synchronize()
         barrier(world)
         torch.cuda.synchronize()
         ev0.record(stream)
-        for i in range(args.steps):
-            step_graphs[i % nsets].replay()
+        run_steps(args.steps)
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -466,7 +474,8 @@ def run_sharq(args, rank, world, local):
         "config": {"workload": f"llama31_8b_qkv_prefill T={T} K={K} N={N} nvfp4 2:4-pairs fused-rmsnorm",
                    "parallelism": f"replicas x{world}" if world > 1 else "single",
                    "l2": f"{nsets} rotating input sets ({nsets * footprint / 2**20:.0f} MiB > L2)",
-                   "launch": "device-timed legs replay one CUDA graph per step; e2e calls the API eagerly"},
+                   "launch": f"device-timed steps replay a CUDA graph of {nsets} consecutive steps (one per "
+                             "input set; a one-step graph per leftover step); e2e calls the API eagerly"},
         "eff_fp4_tflops": eff_tflops, "prep_gbs": prep_gbs,
         "t_prep_us": t_prep_ms * 1e3, "t_linear_us": t_lin_ms * 1e3,
         "roofline": dominant, "roofline_prep": rf_prep, "roofline_gemm": rf_gemm,

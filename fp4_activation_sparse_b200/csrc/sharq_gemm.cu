@@ -81,13 +81,15 @@ struct Stage {
 };
 constexpr int kMaxStageBytes = 52224;  // NVFP4 SharQ: 29696 + 22528
 // bf16 output staging for the epilogue's bulk tensor stores: per epilogue warp one box of 32
-// rows x 32 columns (64-byte rows, 64-byte swizzle), reused four times per tile
+// rows x 32 columns (64-byte rows, 64-byte swizzle), reused four times per tile (on a pair's
+// last tile the boxes go to the then idle pipeline stages instead, four per warp)
 constexpr int kStageOutBytes = 2048;
 constexpr int kOutOffset = kStages * kMaxStageBytes;  // 1024-aligned
 constexpr int kSmemBytes = kOutOffset + kEpiWarps * kStageOutBytes + 1024 /*align slack*/ + 256 /*barriers*/;
 static_assert(Stage<false, true>::kBytes <= kMaxStageBytes && Stage<true, true>::kBytes <= kMaxStageBytes, "stage");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 static_assert(kOutOffset % 1024 == 0, "staging alignment");
+static_assert(4 * kEpiWarps * kStageOutBytes <= kOutOffset, "last-tile boxes fit in the pipeline stages");
 
 struct __align__(64) TmaMaps {
   CUtensorMap act, w;  // both: rows of 1024 bytes (256 x u32), one box = one chunk
@@ -209,6 +211,12 @@ __device__ __forceinline__ void tc_commit_both(uint32_t bar) {
       : "memory");
 }
 
+// L2 prefetch of the 2-D box at (c0, c1) of a tensor map (no shared memory, no completion)
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap *map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // 2-D bulk tensor store from this CTA's shared memory (completion tracked by bulk groups)
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(c0),
@@ -216,9 +224,8 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t sr
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// wait until the committed stores have finished reading shared memory / have completed
+// wait until the committed stores have finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // generic-proxy shared-memory writes become visible to the bulk-copy (async) proxy
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -400,6 +407,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync();  // barriers initialized and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (warp == 0 && lane == 0 && pair < num_tiles) {
+    // The packed weight is not an output of the preparation: its first K steps for this CTA's
+    // first tile are fetched into L2 while the preparation may still be running.
+    const int g = group_of<MAXG>(p, pair), lt = pair - p.grp[g].tile_begin;
+    const int w_row0 = ((lt / p.grp[g].num_m) * BN / 128 + (int)rank) * num_k * (L::W.bytes / 1024);
+    for (int kt = 0; kt < kStages && kt < num_k; ++kt) tma_prefetch_l2(&ms.m[g].w, 0, w_row0 + kt * (L::W.bytes / 1024));
+  }
   // Launched as a programmatic dependent of the preparation: the prologue above overlaps its
   // tail; its outputs are read only after it has completed and flushed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -555,9 +569,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_leader);
       } else {
-        // bf16 output: this warp's 32 rows x 128 columns are read and rounded first (64
-        // registers of packed pairs), the tensor memory is handed back, and the stores
-        // overlap the next tile's MMAs
+        // bf16 output: this warp's 32 rows x 128 columns are read and rounded (64 registers
+        // of packed pairs), the tensor memory is handed back as soon as the last load has
+        // landed, and the stores overlap the next tile's MMAs
         uint32_t packed[4][16];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // two loads in flight per wait
@@ -567,6 +581,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
           reg_fence32(r[0]);
           reg_fence32(r[1]);
+          if (h == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_leader);
+          }
 #pragma unroll
           for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -581,20 +600,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               packed[2 * h + c][i] = *reinterpret_cast<const uint32_t *>(&v);
             }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_leader);
         // Write this warp's 32 x 128 block with bulk tensor stores (coalesced; rows >= T and
-        // columns >= N clipped by the tensor map) through a 2 KB staging box of 32 x 32, in
+        // columns >= N clipped by the tensor map) through 2 KB staging boxes of 32 x 32, in
         // 64-byte-swizzled rows: 16-byte unit u of row r at u ^ ((r / 2) % 4), conflict-free.
+        // One box buffer per warp while MMAs may still read the pipeline stages; on the pair's
+        // last tile every MMA has completed, so the stages' shared memory holds four boxes per
+        // warp and the stores go out back to back.
         const int row0 = m0 + quarter * 32;
+        const bool last = tile + num_pairs >= num_tiles;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          if (lane == 0) bulk_wait_read();  // the previous box has been read out of the buffer
-          __syncwarp();
+          const uint32_t box = last ? smem0 + (uint32_t)(((warp - 2) * 4 + c) * kStageOutBytes) : out_smem;
+          if (!last) {
+            if (lane == 0) bulk_wait_read();  // the previous box has been read out of the buffer
+            __syncwarp();
+          }
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const uint32_t dst = out_smem + lane * 64 + ((u ^ ((lane >> 1) & 3)) << 4);
+            const uint32_t dst = box + lane * 64 + ((u ^ ((lane >> 1) & 3)) << 4);
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(packed[c][4 * u]),
                          "r"(packed[c][4 * u + 1]), "r"(packed[c][4 * u + 2]), "r"(packed[c][4 * u + 3])
                          : "memory");
@@ -602,14 +625,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           fence_proxy_async();
           __syncwarp();
           if (lane == 0) {
-            if (row0 < G.T && col0 + 32 * c < p.N) tma_store_2d(&ms.m[g].y, out_smem, col0 + 32 * c, row0);
+            if (row0 < G.T && col0 + 32 * c < p.N) tma_store_2d(&ms.m[g].y, box, col0 + 32 * c, row0);
             bulk_commit();
           }
         }
       }
       acc_phase ^= 1u;
     }
-    if (lane == 0) bulk_wait_all();  // the output stores have completed before the CTA exits
+    // the stores have read their boxes before the CTA's shared memory goes away (they complete
+    // in global memory before the grid does)
+    if (lane == 0) bulk_wait_read();
   }
 
   else {
@@ -670,6 +695,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   // Both CTAs: the leader arrives here only after its MMAs drained, so neither CTA frees
   // tensor memory the pair's MMAs still write, and no remote arrive targets an exited CTA.
+  // The roles above run on lane 0 of their warps: each warp converges before the aligned
+  // cluster barrier.
+  __syncwarp();
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
