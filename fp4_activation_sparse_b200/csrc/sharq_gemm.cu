@@ -29,12 +29,14 @@
 //               the tensor's edges) while the next tile's MMAs run. Row-wise 16-byte stores
 //               from registers took a quarter of the kernel's time and delayed the next tile's
 //               loads. (float32 output, a test format, is stored from registers.)
-//   warps 10-14 scale copiers (leader): tcgen05.cp of the K step's scales and metadata into one
-//               of three tensor-memory buffers, split five ways (dense-view weight scales of
-//               the first and second K halves, sparse-view weight scales, residual scales,
-//               backbone scales + metadata), each from its own thread: a copy costs its
-//               issuing thread tens of cycles, so the copies keep pace with the MMAs only
-//               when spread over several threads.
+//   warps 10-13 scale writers (both CTAs, one tensor-memory lane quarter each): the K step's
+//               scales and metadata from shared memory into registers and with tcgen05.st into
+//               one of three tensor-memory buffers (every quarter holds each 32-row scale atom,
+//               the layout the block-scaled MMA reads). tcgen05.cp copies issued by the leader
+//               did the same but ran in order with the MMAs in the tensor pipe (~930 cycles
+//               per K step against 768 of MMA work); the stores keep that pipe for the MMAs.
+//               Each CTA's loads complete on its own stage barrier; the leader's MMA thread
+//               waits for the writers of both CTAs.
 // One launch may cover several problems of the same N and K (the experts of a mixture-of-
 // experts layer): the persistent loop decodes each pair tile into (group, m-block, n-block)
 // from a prefix table of tile counts. The kernel is launched as a programmatic dependent of
@@ -60,8 +62,8 @@ constexpr int BN = 256;   // output columns per pair tile
 constexpr int BK = 256;   // logical K per stage
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;
-constexpr int kCopiers = 5;
-constexpr int kThreads = 64 + 32 * kEpiWarps + 32 * kCopiers;  // producer, MMA, epilogue, scale copiers
+constexpr int kSfWarps = 4;  // one per tensor-memory lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps + 32 * kSfWarps;  // producer, MMA, epilogue, scale writers
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = 256;
 constexpr uint32_t kScaleBufCols = 80;  // per buffer: meta 4, SFA_sp 8, SFA_res 16, SFB_sp 16, SFB_res 32
@@ -182,12 +184,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
   }
 }
 
-__device__ __forceinline__ void spin_ns(uint64_t ns) {
-  const uint64_t t0 = globaltimer();
-  while (globaltimer() - t0 < ns) {
-  }
-}
-
 // 2-D TMA load into this CTA's shared memory, completing on the barrier at `bar_cluster`
 // (the leader CTA's barrier) -- the cta_group::2 form lets either CTA of the pair signal it.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
@@ -229,15 +225,6 @@ __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.w
 // generic-proxy shared-memory writes become visible to the bulk-copy (async) proxy
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// arrive once on the leader CTA's barrier at this offset when this thread's tcgen05 operations finish
-__device__ __forceinline__ void tc_commit_leader(uint32_t bar) {
-  const uint16_t mask = 0x1;
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
-      "h"(mask)
-      : "memory");
-}
-
 // Shared-memory matrix descriptors (K-major) as templates with the address field zero;
 // layout 0 none, 2 SW128, 4 SW64; bit 46 is the sm_100 descriptor version. dsc() adds the
 // 16-byte-unit address of one operand.
@@ -247,7 +234,6 @@ constexpr uint64_t desc_template(uint32_t sbo_bytes, uint32_t layout, uint32_t l
 }
 constexpr uint64_t kDescSw128 = desc_template(1024, 2, 16);  // 8-row groups of 128 B
 constexpr uint64_t kDescSw64 = desc_template(512, 4, 16);    // 8-row groups of 64 B
-constexpr uint64_t kDescNone = desc_template(128, 0, 0);     // 8 rows x 16 B core matrices
 __device__ __forceinline__ uint64_t dsc(uint64_t tmpl, uint32_t addr16) { return tmpl | (uint64_t)(addr16 & 0x3FFFu); }
 
 // Instruction descriptor of the block-scaled MMA kinds (mxf4 / mxf4nvf4): E2M1 A and B,
@@ -298,17 +284,6 @@ __device__ __forceinline__ void mma_sparse(uint32_t d_tmem, uint64_t a, uint64_t
         "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb), "r"(meta));
 }
 
-// 32 rows x 128 bits (one 512-byte scale atom), replicated into the four lane quarters;
-// issued by the leader, performed in both CTAs from their own shared memory.
-__device__ __forceinline__ void tc_cp_atom(uint32_t taddr, uint64_t desc) {
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
-}
-
-// 128 rows x 128 bits (metadata of 256 logical K), in both CTAs.
-__device__ __forceinline__ void tc_cp_128x128(uint32_t taddr, uint64_t desc) {
-  asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
-}
-
 // 32 lanes x 32 columns of 32 bits; asynchronous until tmem_ld_wait()
 __device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t *r) {
   asm volatile(
@@ -322,6 +297,47 @@ __device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t *r) {
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x N columns of 32 bits from registers (lane l writes r[0..N) to its lane)
+__device__ __forceinline__ void tmem_st_x4(uint32_t taddr, const uint32_t *r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t *r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t *r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t *r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+               : "memory");
+}
+template <int N>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t *r) {
+  if (N == 4) tmem_st_x4(taddr, r);
+  if (N == 8) tmem_st_x8(taddr, r);
+  if (N == 16) tmem_st_x16(taddr, r);
+  if (N == 32) tmem_st_x32(taddr, r);
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// NA scale atoms (32 rows x 16 bytes each, at smem addresses base + atom_off(i)) into NA
+// groups of 4 consecutive tensor-memory columns of this warp's lane quarter: lane l writes row
+// l of every atom, so each quarter holds the whole atom (the replicated layout of the block-
+// scaled MMA's scale factors).
+template <int NA, typename F>
+__device__ __forceinline__ void st_atoms(uint32_t taddr, uint32_t base, F atom_off, int lane) {
+  uint32_t r[4 * NA];
+#pragma unroll
+  for (int i = 0; i < NA; ++i)
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[4 * i]), "=r"(r[4 * i + 1]), "=r"(r[4 * i + 2]), "=r"(r[4 * i + 3])
+                 : "r"(base + atom_off(i) + lane * 16));
+  tmem_st<4 * NA>(taddr, r);
+}
 
 // Orders every later use of r after the preceding tmem_ld_wait(): the registers written by
 // an asynchronous tensor-memory load are only valid once the wait has returned.
@@ -355,9 +371,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOutOffset + kEpiWarps * kStageOutBytes);
-  // bars: full[kStages], empty[kStages], acc_full, acc_empty, drain, sf_full[kStages], sf_free[kScaleBufs],
-  // sf_drain[kCopiers]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 3 + kScaleBufs + kCopiers);
+  // bars: full[kStages], empty[kStages], acc_full, acc_empty, drain, sf_full[kStages], sf_free[kScaleBufs]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 3 + kScaleBufs);
   volatile uint32_t *abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -370,7 +385,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t acc_full = bar0 + 8u * (2 * kStages), acc_empty = acc_full + 8, drain_bar = acc_full + 16;
   auto sf_full_bar = [&](int s) { return bar0 + 8u * (2 * kStages + 3 + s); };
   auto sf_free_bar = [&](uint32_t b) { return bar0 + 8u * (3 * kStages + 3 + b); };
-  auto sf_drain_bar = [&](int c) { return bar0 + 8u * (3 * kStages + 3 + kScaleBufs + c); };
 
   using L = Stage<MX, SPARSE>;
   constexpr int apt_res = atoms_res(MX ? 1 : 0), apt_sp = atoms_sp(MX ? 1 : 0);
@@ -388,9 +402,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kEpiWarps);
     mbar_init(drain_bar, 1);
-    for (int s = 0; s < kStages; ++s) mbar_init(sf_full_bar(s), kCopiers);  // one commit per copier
+    for (int s = 0; s < kStages; ++s) mbar_init(sf_full_bar(s), 2 * kSfWarps);  // writers of both CTAs
     for (uint32_t b = 0; b < kScaleBufs; ++b) mbar_init(sf_free_bar(b), 1);
-    for (int c = 0; c < kCopiers; ++c) mbar_init(sf_drain_bar(c), 1);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -424,8 +437,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, last_parity = 0;  // bit s: stage s armed / its last phase parity
-      bool issued = false, ok = true;
-      const uint32_t full_leader0 = map_to_rank(full_bar(0), 0);
+      bool ok = true;
+      const uint32_t full_own0 = map_to_rank(full_bar(0), rank);
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
         const int g = group_of<MAXG>(p, tile), lt = tile - p.grp[g].tile_begin, num_m = p.grp[g].num_m;
         const TmaMaps &maps = ms.m[g];
@@ -436,30 +449,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int kt = 0; kt < num_k; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, limit, abort_flag)) { ok = false; break; }
           const uint32_t st = smem0 + stage * kStageBytes;
-          if (leader) {
-            mbar_expect_tx(full_bar(stage), 2u * kStageBytes);
-            armed |= 1u << stage;
-            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          }
-          const uint32_t fb = full_leader0 + 8u * stage;
+          // each CTA's loads complete on its own barrier: its scale writers wait for it, and
+          // the leader's MMA learns of the peer's bytes through the peer's writers
+          mbar_expect_tx(full_bar(stage), kStageBytes);
+          armed |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          const uint32_t fb = full_own0 + 8u * stage;
           tma_load_2d(st, &maps.act, 0, a_row0 + kt * (L::A.bytes / 1024), fb);
           tma_load_2d(st + L::kW, &maps.w, 0, w_row0 + kt * (L::W.bytes / 1024), fb);
-          issued = true;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
       if (!ok) {
-        // Drain before exit: the leader sees every phase it armed complete (its own and the
-        // peer's bytes); the peer cannot observe the leader's barrier, so it lets its loads land.
-        if (leader) {
-          for (int s = 0; s < kStages; ++s)
-            if (armed & (1u << s)) {
-              volatile uint32_t no_abort = 0;
-              mbar_wait(full_bar(s), (last_parity >> s) & 1u, kDrainLimitNs, &no_abort);
-            }
-        } else if (issued) {
-          spin_ns(200000);
-        }
+        // Drain before exit: every phase this CTA armed completes (its loads have landed).
+        for (int s = 0; s < kStages; ++s)
+          if (armed & (1u << s)) {
+            volatile uint32_t no_abort = 0;
+            mbar_wait(full_bar(s), (last_parity >> s) & 1u, kDrainLimitNs, &no_abort);
+          }
       }
     }
   } else if (warp == 1) {
@@ -474,8 +481,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!mbar_wait<true>(acc_empty, acc_phase ^ 1u, limit, abort_flag)) { ok = false; break; }
         tc_fence_after();
         for (int kt = 0; kt < num_k; ++kt) {
-          // the scale copiers waited for this stage's bytes before copying its scales
-          if (!mbar_wait(sf_full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
+          // the scale writers of both CTAs waited for their stage's bytes, then wrote its scales
+          // (remote arrives: cluster-scope acquire)
+          if (!mbar_wait<true>(sf_full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
           if (!mbar_wait(full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
           tc_fence_after();
           // descriptors: constant templates plus the operand's shared-memory address >> 4
@@ -509,7 +517,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             accumulate = 1u;
           }
           tc_commit_both(empty_bar(stage));  // frees the stage in both CTAs once these MMAs have read it
-          tc_commit_leader(sf_free_bar(buf));  // and the scale buffer
+          tc_commit_both(sf_free_bar(buf));  // and the scale buffer in both CTAs
           if (++buf == kScaleBufs) buf = 0;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
@@ -638,58 +646,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 
   else {
-    // ------------------------------------------------------------ scale copiers (warps 10..14; leader)
-    const int which = warp - (2 + kEpiWarps);
-    if (lane == 0 && leader) {
-      int stage = 0;
-      uint32_t phase = 0, buf = 0, buf_phase = 0;
-      bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        for (int kt = 0; kt < num_k; ++kt) {
-          if (!mbar_wait(full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
-          // the buffer is free once the MMAs that last read it (kScaleBufs steps ago) completed
-          if (!mbar_wait(sf_free_bar(buf), buf_phase ^ 1u, limit, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t st4 = (smem0 + stage * kStageBytes) >> 4;
-          const uint32_t sbuf = tmem + kAccCols + buf * kScaleBufCols;
-          const uint32_t t_meta = sbuf, t_sfa_sp = sbuf + 4, t_sfa_res = sbuf + 12, t_sfb_sp = sbuf + 28,
-                         t_sfb_res = sbuf + 44;
-          constexpr int kA = 0, kW = L::kW;
-          // shared memory -> tensor memory (both CTAs). The weight chunk holds the scales of
-          // both 128-row halves of the pair's 256 columns.
-          if (which < 2) {  // dense-view weight scales, one K half each (both 128-row n-blocks)
-#pragma unroll
-            for (int a = which * apt_res / 2; a < (which + 1) * apt_res / 2; ++a) {
-              tc_cp_atom(t_sfb_res + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_res + a * 512) / 16));
-              tc_cp_atom(t_sfb_res + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_res + (apt_res + a) * 512) / 16));
-            }
-          } else if (which == 2) {  // sparse-view weight scales
-            if (SPARSE) {
-#pragma unroll
-              for (int a = 0; a < apt_sp; ++a) {
-                tc_cp_atom(t_sfb_sp + 8 * a, dsc(kDescNone, st4 + (kW + L::W.sf_sp + a * 512) / 16));
-                tc_cp_atom(t_sfb_sp + 8 * a + 4, dsc(kDescNone, st4 + (kW + L::W.sf_sp + (apt_sp + a) * 512) / 16));
-              }
-            }
-          } else if (which == 3) {  // residual scales
-#pragma unroll
-            for (int a = 0; a < apt_res; ++a)
-              tc_cp_atom(t_sfa_res + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_res + a * 512) / 16));
-          } else if (SPARSE) {  // backbone scales and metadata
-#pragma unroll
-            for (int a = 0; a < apt_sp; ++a)
-              tc_cp_atom(t_sfa_sp + 4 * a, dsc(kDescNone, st4 + (kA + L::A.sf_sp + a * 512) / 16));
-            tc_cp_128x128(t_meta, dsc(kDescNone, st4 + (kA + L::A.meta) / 16));
-          }
-          tc_commit_leader(sf_full_bar(stage));
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
-          if (++buf == kScaleBufs) { buf = 0; buf_phase ^= 1u; }
+    // ------------------------------------------------------------ scale writers (warps 10..13, both CTAs)
+    // Each warp writes the K step's scale factors and metadata into its lane quarter of one of
+    // three tensor-memory buffers with tcgen05.st (registers -> tensor memory), so these writes
+    // stay out of the tensor pipe that runs the MMAs in order.
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const uint32_t sf_full_leader0 = map_to_rank(sf_full_bar(0), 0);
+    int stage = 0;
+    uint32_t phase = 0, buf = 0, buf_phase = 0;
+    bool ok = true;
+    for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+      for (int kt = 0; kt < num_k; ++kt) {
+        if (!mbar_wait(full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
+        // the buffer is free once the MMAs that last read it (kScaleBufs steps ago) completed
+        if (!mbar_wait(sf_free_bar(buf), buf_phase ^ 1u, limit, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = smem0 + stage * kStageBytes;
+        const uint32_t sbuf = tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols + buf * kScaleBufCols;
+        const uint32_t t_meta = sbuf, t_sfa_sp = sbuf + 4, t_sfa_res = sbuf + 12, t_sfb_sp = sbuf + 28,
+                       t_sfb_res = sbuf + 44;
+        constexpr int kA = 0, kW = L::kW;
+        // weight scales: the chunk holds the atoms of both 128-row halves of the pair's 256
+        // columns (half 0, then half 1); in tensor memory they alternate per atom
+        st_atoms<2 * apt_res>(t_sfb_res, st + kW + L::W.sf_res,
+                              [&](int i) { return ((i & 1) * apt_res + (i >> 1)) * 512; }, lane);
+        if (SPARSE)
+          st_atoms<2 * apt_sp>(t_sfb_sp, st + kW + L::W.sf_sp,
+                               [&](int i) { return ((i & 1) * apt_sp + (i >> 1)) * 512; }, lane);
+        st_atoms<apt_res>(t_sfa_res, st + kA + L::A.sf_res, [&](int i) { return i * 512; }, lane);
+        if (SPARSE) {
+          st_atoms<apt_sp>(t_sfa_sp, st + kA + L::A.sf_sp, [&](int i) { return i * 512; }, lane);
+          // metadata: 128 rows x 16 bytes, row r in lane r (not replicated)
+          st_atoms<1>(t_meta, st + kA + L::A.meta + quarter * 32 * 16, [&](int) { return 0; }, lane);
         }
+        // The stores have completed in this SM's tensor memory (wait::st) before the arrive
+        // leaves; the MMA that reads them is issued only after the leader has seen all eight
+        // arrives. Nothing in the memory hierarchy sits between the two, so the arrive is
+        // relaxed: a cluster-scope release arrive stalled each writer ~1400 cycles per K step,
+        // which made the writers, not the MMAs, set the pace (54 us against 35 us per launch).
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_relaxed(sf_full_leader0 + 8u * stage);
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        if (++buf == kScaleBufs) { buf = 0; buf_phase ^= 1u; }
       }
-      // Drain: the copies issued above complete before TMEM is released.
-      tc_commit_leader(sf_drain_bar(which));
-      volatile uint32_t no_abort = 0;
-      mbar_wait(sf_drain_bar(which), 0, kDrainLimitNs, &no_abort);
     }
   }
 
