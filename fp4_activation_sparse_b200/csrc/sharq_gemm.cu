@@ -16,7 +16,7 @@
 // two bulk tensor copies per CTA -- the copy count per stage, not the bytes, is what
 // bounds a TMA-fed pipeline at this tile size.
 //   warp 0      TMA producer (both CTAs): the activation chunk and the weight chunk of the
-//               K step; every load completes on the leader CTA's barrier.
+//               K step; each CTA's loads complete on its own stage barrier.
 //   warp 1      TMEM owner (both CTAs) and, in the leader, the single MMA-issuing thread:
 //               two tcgen05.mma.sp (K=128 logical, pairwise 4:8) and four dense tcgen05.mma
 //               (K=64) per K step accumulate into one fp32 accumulator of 128 x 256 per CTA.
@@ -184,8 +184,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
   }
 }
 
-// 2-D TMA load into this CTA's shared memory, completing on the barrier at `bar_cluster`
-// (the leader CTA's barrier) -- the cta_group::2 form lets either CTA of the pair signal it.
+// 2-D TMA load into this CTA's shared memory, completing on the barrier at `bar_cluster` (a
+// shared::cluster address; the kernel passes this CTA's own stage barrier).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
                                             uint32_t bar_cluster) {
   asm volatile(
