@@ -150,3 +150,27 @@ def test_linear_full_size_sampled_outputs(which):
     got = hw.to_np(y)[np.ix_(rows, cols)]
     max_abs, frob = gemm_errors(got, ref)
     assert max_abs <= MAX_ABS_TOL and frob <= FROB_TOL, (max_abs, frob)
+
+
+def test_linear_full_size_every_output():
+    """The benchmark's GEMM launch (Llama-3.1-8B QKV, 2048 x 4096 -> 6144: 192 pair tiles on
+    every SM pair) against the oracle on all 12.6 M outputs, float32 and bf16: every tile of
+    every wave, including tiles whose scale buffers were handed between the two CTAs of a
+    pair thousands of times."""
+    S = require_gpu()
+    lin = wl.llama_qkv(T=2048)
+    x = to_dev_bf16(lin.x)
+    wp = S.sharq_pack_weight(to_dev_bf16(lin.w), 0)
+    p = S.sharq_prepare(x, None, lin.eps, 2, 4, 2, 0)
+    y32 = S.sharq_linear(p, wp, out_dtype=torch.float32)
+    y16 = S.sharq_linear(p, wp)
+    torch.cuda.synchronize()
+    assert S.sharq_device_status() == S.SHARQ_OK
+    ref = O.linear(O.prepare(f32(lin.x), None, lin.eps, 2, 4, 2, O.NVFP4), O.pack_weight(f32(lin.w), O.NVFP4))
+    got = hw.to_np(y32)
+    max_abs, frob = gemm_errors(got, ref)
+    assert max_abs <= MAX_ABS_TOL and frob <= FROB_TOL, (max_abs, frob)
+    # per-tile check: no 256 x 256 output tile may carry a large share of the error
+    tile_err = np.abs(got - ref).reshape(8, 256, 24, 256).max(axis=(1, 3)) / np.abs(ref).max()
+    assert tile_err.max() <= MAX_ABS_TOL, np.argwhere(tile_err > MAX_ABS_TOL)[:5]
+    assert torch.equal(y16, y32.to(torch.bfloat16))
