@@ -184,6 +184,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
   }
 }
 
+// The same wait in every lane of a warp, with a vote: the warp goes on only if every lane's
+// wait succeeded, so it stays converged for the aligned tcgen05 instructions that follow even
+// if lanes reached the time limit differently.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                               volatile uint32_t *abort_flag) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, limit_ns, abort_flag)) != 0;
+}
+
 // 2-D TMA load into this CTA's shared memory, completing on the barrier at `bar_cluster` (a
 // shared::cluster address; the kernel passes this CTA's own stage barrier).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
@@ -545,7 +553,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int m0 = (lt % num_m) * (2 * BM) + (int)rank * BM, n0 = (lt / num_m) * BN;
       const int row = m0 + r_local;
       const float scale = row < G.T ? __fmul_rn(G.row_scale[row], s_w) : 0.f;
-      if (!mbar_wait(acc_full, acc_phase, limit, abort_flag)) break;
+      if (!mbar_wait_warp(acc_full, acc_phase, limit, abort_flag)) break;
       tc_fence_after();
       const uint32_t tacc = tmem + ((uint32_t)(quarter * 32) << 16) + col_half * 128;
       const int col0 = n0 + col_half * 128;
@@ -657,9 +665,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
       for (int kt = 0; kt < num_k; ++kt) {
-        if (!mbar_wait(full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
         // the buffer is free once the MMAs that last read it (kScaleBufs steps ago) completed
-        if (!mbar_wait(sf_free_bar(buf), buf_phase ^ 1u, limit, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(sf_free_bar(buf), buf_phase ^ 1u, limit, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = smem0 + stage * kStageBytes;
         const uint32_t sbuf = tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols + buf * kScaleBufCols;
