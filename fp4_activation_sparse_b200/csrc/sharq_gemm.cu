@@ -69,7 +69,7 @@ constexpr uint32_t kAccCols = 256;
 constexpr uint32_t kScaleBufCols = 80;  // per buffer: meta 4, SFA_sp 8, SFA_res 16, SFB_sp 16, SFB_res 32
 constexpr uint32_t kScaleBufs = 3;      // 256 + 3 * 80 = 496 of 512 columns
 static_assert(kAccCols + kScaleBufs * kScaleBufCols <= kTmemCols, "tensor memory");
-// Drains (own copies and MMAs in flight before exit) always get the full bound, also when a
+// Drains (own bulk copies and MMAs in flight before exit) always get the full bound, also when a
 // test lowers the limit of the ordinary waits.
 constexpr uint64_t kDrainLimitNs = 4000000000ull;
 
@@ -533,7 +533,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_commit_both(acc_full);
         acc_phase ^= 1u;
       }
-      // Drain: all MMAs and copies issued above complete before TMEM is released.
+      // Drain: all MMAs issued above complete before TMEM is released.
       tc_commit_both(drain_bar);
       volatile uint32_t no_abort = 0;
       mbar_wait(drain_bar, 0, kDrainLimitNs, &no_abort);
