@@ -202,6 +202,11 @@ def blas_threads():
         return os.cpu_count()
 
 
+def host_cores() -> dict:
+    """Cores of the host the oracle runs on: all logical CPUs and the BLAS pool's threads."""
+    return {"os_cpu_count": os.cpu_count(), "blas_threads": blas_threads()}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -217,7 +222,8 @@ def run_reference(args, rank, world):
         "data": "synthetic (seeded outlier-channel activations, N(0,0.02) weight)",
         "config": {"workload": f"llama31_8b_qkv_prefill T={T} K={K} N={N} nvfp4 2:4-pairs fused-rmsnorm",
                    "rows_per_step": rows},
-        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "host_cores": host_cores(),
+                         "kind": "oracle",
                          "sample": f"{rows} token rows per step x {args.steps} steps (prep + float64 GEMM vs all "
                                    f"{N} outputs); weight packed once outside timing"},
         "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -499,7 +505,8 @@ def run_sharq(args, rank, world, local):
     }
     if world == 1 and not args.no_cpu_baseline:
         tps, secs, done = oracle_throughput(lin, 128, 8, 1)
-        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(),
+                                "host_cores": host_cores(), "kind": "oracle",
                                 "sample": f"8 steps x 128 token rows (prep + float64 GEMM vs all {N} outputs), "
                                           f"{secs:.1f} s"}
     print(json.dumps(line), flush=True)

@@ -1,6 +1,7 @@
 // C ABI of the SharQ library: argument checks, buffer sizes, launches.
 // Every entry point validates on the host before it launches anything and returns a
 // sharq_status; the message of the last failure is kept per host thread.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -12,7 +13,9 @@
 namespace {
 
 thread_local char g_err[512] = "";
-long long g_wait_limit = 0;
+// Time limit (ns) of the GEMM's bounded waits for calls issued from now on, process-wide;
+// 0 = the kernel's default. Read once per launch.
+std::atomic<long long> g_wait_limit{0};
 
 int fail(int status, const char *fmt, ...) {
   va_list ap;
@@ -55,7 +58,7 @@ const char *sharq_last_error(void) { return g_err; }
 
 int sharq_version(void) { return 200; }
 
-void sharq_set_wait_limit(long long spins) { g_wait_limit = spins; }
+void sharq_set_wait_limit(long long nanoseconds) { g_wait_limit.store(nanoseconds, std::memory_order_relaxed); }
 
 size_t sharq_prep_buffer_sizes(int tokens, int k, int nm_n, int nm_m, int unit, int fmt, size_t sizes[2]) {
   if (!sizes) { fail(SHARQ_ERR_INVALID_ARG, "sizes is null"); return 0; }
@@ -209,7 +212,7 @@ static int check_wpack(const sharq_wpack *w) {
 }
 
 static int run_gemm(sharq::GemmParams &g, const char *name, cudaStream_t st) {
-  g.wait_limit = g_wait_limit;
+  g.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
   const char *why = nullptr;
   cudaError_t e = sharq::launch_gemm(g, st, &why);
   if (why) return fail(SHARQ_ERR_CUDA, "%s: %s", name, why);
@@ -268,7 +271,7 @@ int sharq_linear_grouped(const sharq_prep *a, const sharq_wpack *w, void *const 
   if (!a || !w || !y) return fail(SHARQ_ERR_INVALID_ARG, "null group arrays");
   if (n_groups < 1) return fail(SHARQ_ERR_INVALID_ARG, "n_groups must be >= 1 (got %d)", n_groups);
   for (int e = 0; e < n_groups; ++e) {
-    if (a[e].tokens == 0 && y[e]) continue;  // an expert without tokens: nothing to do
+    if (a[e].tokens == 0) continue;  // an expert without tokens: nothing to do (y[e] may be null)
     if (int s = check_linear(&a[e], &w[e], y[e], out_dtype)) return s;
     if (w[e].n_out != w[0].n_out || w[e].k != w[0].k || w[e].fmt != w[0].fmt)
       return fail(SHARQ_ERR_INVALID_ARG, "group %d: every weight must have the shape and format of group 0", e);

@@ -1,11 +1,11 @@
 // SharQ linear layer GEMM (K3): structured-sparse + dense block-scaled FP4 MMAs into one
 // tensor-memory accumulator, one epilogue.
 //
-// "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM Inference",
-// Abstract: "A sparse FP4 GEMM processes the backbone while a dense FP4 GEMM
-// compensates for both mask-induced activation loss and sparse-path quantization
-// error. The two paths share a single FP4 weight payload with path-specific scale
-// views." The README ("Benchmarks") enables "epilogue fusion" on this path.
+// Per "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM Inference"
+// (Abstract), the backbone goes through a sparse FP4 GEMM and the residual through a
+// dense FP4 GEMM that makes up for what the mask dropped and for the backbone's
+// quantization error; both read the same FP4 weight codes, each path with its own
+// scale view. The README mirror ("Benchmarks") runs this path with the epilogue fused.
 //
 // sm_100a design. A cluster of two CTAs on the two SMs of a TPC works on one 256 x 256
 // output tile with cta_group::2 MMAs (M = 256, N = 256): each CTA loads its own 128

@@ -1,8 +1,8 @@
 // Weight packer (K1): one FP4 weight payload with path-specific scale views.
 //
-// "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM Inference",
-// Abstract: "The two paths share a single FP4 weight payload with path-specific
-// scale views." The weight is quantized once, in blocks of 2B consecutive K
+// Per "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM Inference"
+// (Abstract), the sparse and the dense path read one set of FP4 weight codes, each with
+// scales laid out for its own MMA. The weight is quantized once, in blocks of 2B consecutive K
 // positions (B = 16 NVFP4 / 32 MXFP4): that is the K span one scale covers in the
 // structured-sparse block-scaled MMA, whose scale vector counts stored values of a
 // 50%-dense operand. The dense MMA needs one scale per B positions, so its view

@@ -1,17 +1,16 @@
 /*
  * sharq.h -- C ABI of the SharQ sparse-dense FP4 linear layer for B200 (sm_100a).
  *
- * The method ("SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM
- * Inference", Abstract): an online sparse-dense decomposition of each activation
- * tensor. An input-adaptive N:M mask extracts an outlier-dominated sparse
- * backbone, the backbone is quantized to FP4, a dense residual is defined
- * against the *quantized* backbone and quantized densely to FP4; a sparse FP4
- * GEMM on the backbone and a dense FP4 GEMM on the residual share one FP4
- * weight payload with path-specific scale views; a fused preparation kernel
- * absorbs mask generation, residual construction and layer normalization.
- * The README ("SharQ: Bridging Activation Sparsity and FP4 Quantization",
- * sections "Evaluation" and "Benchmarks") names the normalization RMSNorm and
- * the dense-FP4-only mode "NVFP4".
+ * The method follows "SharQ: Bridging Activation Sparsity and FP4 Quantization for
+ * LLM Inference" (Abstract). Every activation tensor is split at run time into two
+ * FP4 operands: a structured-sparse one holding the N largest of every M values
+ * along K (where the outliers end up), and a dense remainder computed against the
+ * backbone *after* its FP4 rounding. The sparse operand feeds a sparse FP4 MMA, the
+ * remainder a dense FP4 MMA; both multiply the same FP4 weight codes, each with its
+ * own scale layout, and add into one output. Normalization, mask selection and both
+ * quantizations happen in one preparation kernel. The README mirror ("SharQ:
+ * Bridging Activation Sparsity and FP4 Quantization", sections "Evaluation" and
+ * "Benchmarks") names the normalization RMSNorm and calls the dense-only mode NVFP4.
  *
  * Conventions for every call:
  *  - Pointers named *_dev are device pointers; the caller allocates and owns all
@@ -130,17 +129,16 @@ size_t sharq_dense_buffer_sizes(int tokens, int k, int fmt, size_t sizes[2]);
 size_t sharq_wpack_buffer_sizes(int n_out, int k, int fmt, size_t sizes[2]);
 
 /* Pack a bf16 weight once (offline): per-tensor amax, block scales over 2B
- * consecutive K, E2M1 codes, and both scale views. The abstract: "The two paths
- * share a single FP4 weight payload with path-specific scale views."
+ * consecutive K, E2M1 codes, and both scale views (Abstract: the two GEMM paths read
+ * the same weight codes, each with scales laid out for it).
  *   w_bf16_dev  [n_out][k] row-major bf16
  *   out         caller-filled struct of device buffers (fields n_out/k/fmt are set here)
  * Two launches (amax reduction, then quantization); tensor_scale is cleared first. */
 int sharq_pack_weight(const void *w_bf16_dev, int n_out, int k, int fmt, sharq_wpack *out,
                       void *stream);
 
-/* The fused preparation operator (one launch). The abstract: "a fused
- * preparation kernel absorbs mask generation, residual construction, and layer
- * normalization into one operator".
+/* The fused preparation operator (one launch; Abstract: normalization, the mask and the
+ * residual are computed by one kernel).
  *   x_bf16_dev      [tokens][k] row-major bf16 activations
  *   gamma_bf16_dev  [k] bf16 RMSNorm weight, or NULL for no normalization
  *   eps             RMSNorm epsilon (ignored without gamma)
@@ -166,8 +164,8 @@ int sharq_prepare_tensor_scale(const void *x_bf16_dev, int tokens, int k, const 
 
 /* The preparation operator fed by a gate/up projection's output (one launch): the down
  * projection's input x = SiLU(g) * u is formed in registers from [g | u] and prepared as
- * by sharq_prepare without normalization, so x never goes through memory. The abstract's
- * fused preparation kernel "absorbs" the steps in front of the quantizer into one operator.
+ * by sharq_prepare without normalization, so x never goes through memory (the abstract's
+ * preparation kernel folds the steps in front of the quantizer into itself).
  *   gate_up_bf16_dev  [tokens][2k] row-major bf16: g in columns [0, k), u in [k, 2k);
  *                     32-byte aligned
  *   x = bf16(fp32(silu(g) * u)) rounded to nearest even, silu(g) = g * sigma(g) in float32
@@ -194,13 +192,14 @@ int sharq_linear(const sharq_prep *a, const sharq_wpack *w, void *y_dev, int out
  * their own buffers, so no tile mixes experts). The abstract evaluates a mixture-of-experts
  * model (Qwen3-30B-A3B) with the method; this is its expert layer.
  *   a[e], w[e]  prepared activation and packed weight of group e; every weight has the same
- *               n_out, k and fmt; a[e].tokens == 0 marks an expert without tokens (skipped)
+ *               n_out, k and fmt; a[e].tokens == 0 marks an expert without tokens (skipped:
+ *               its prep buffers and y_dev[e] are not used and may be NULL)
  *   y_dev[e]    [a[e].tokens][n_out] output of group e (bf16 or float32 per out_dtype)
  * Checks and errors as sharq_linear, per group. */
 int sharq_linear_grouped(const sharq_prep *a, const sharq_wpack *w, void *const *y_dev, int n_groups,
                          int out_dtype, void *stream);
 
-/* The library's own dense FP4 baseline (the README's "NVFP4: dense FP4 baseline"):
+/* The library's own dense FP4 baseline (the README mirror's dense-only NVFP4 mode):
  * optional RMSNorm + dense block quantization of xh with the same row-scale rule
  * (one launch), and a dense FP4 GEMM against the weight's dense view (one launch).
  *   tiles_dev      dense-quantized activation chunks (sharq_dense_buffer_sizes)
@@ -215,7 +214,8 @@ int sharq_linear_dense(const void *tiles_dev, const float *row_scale_dev, int to
 int sharq_device_status(void *stream);
 
 /* Test hook: time limit, in nanoseconds, of the GEMM's bounded waits (0 restores the
- * default of 4 s). Lowering it lets a test make a wait give up without faulting the device:
+ * default of 4 s). Process-wide (one atomic value shared by every host thread), read by
+ * each GEMM call when it launches. Lowering it lets a test make a wait give up without faulting the device:
  * the kernel records SHARQ_ERR_TIMEOUT, drains its own copies and MMAs, frees its tensor
  * memory and returns; its output is then undefined. Applies to calls issued afterwards. */
 void sharq_set_wait_limit(long long nanoseconds);

@@ -77,8 +77,8 @@ def block_size(fmt: str) -> int:
 def rmsnorm(x: np.ndarray, gamma: np.ndarray | None, eps: float) -> np.ndarray:
     """Layer normalization fused into the preparation operator.
 
-    The abstract says the fused preparation kernel absorbs "layer normalization";
-    the README's benchmark notes (section "Benchmarks") name it RMSNorm fusion.
+    The abstract lists layer normalization among the steps folded into the fused
+    preparation kernel; the README mirror (section "Benchmarks") calls it RMSNorm fusion.
     ``x`` holds the bf16 activations as float32 [T, K]; ``gamma`` the bf16
     weight as float32 [K] or None (no normalization).
     """
@@ -100,8 +100,8 @@ def rmsnorm(x: np.ndarray, gamma: np.ndarray | None, eps: float) -> np.ndarray:
 def nm_select(xh: np.ndarray, n: int, m: int, unit: int) -> np.ndarray:
     """Indices of the kept units: int array [T, G, n], ascending within each group.
 
-    The abstract: "SharQ generates an input-adaptive N:M mask to extract an
-    outlier-dominated sparse backbone". A group is M consecutive units of
+    Per the abstract, a mask chosen from the input itself (N of every M) pulls
+    out a sparse backbone that carries the outliers. A group is M consecutive units of
     ``unit`` elements along K; the N units of largest key survive, key = the
     largest |xh| inside the unit, ties to the lower unit index.
     """
@@ -234,9 +234,9 @@ def _quantize(vals2d: np.ndarray, fmt: str, s_x, g_x):
 def prepare(x, gamma, eps: float, n: int, m: int, unit: int, fmt: str, per_tensor: bool = False) -> dict:
     """SharQ's fused preparation operator, written out step by step.
 
-    Abstract: mask -> backbone -> "quantizes it to FP4" -> "defines a dense
-    residual relative to the quantized sparse backbone rather than the
-    unquantized sparse values" -> dense FP4 of that residual.
+    Order of the abstract: mask -> backbone -> FP4 backbone -> residual taken
+    against the backbone after quantization (not against its exact values) ->
+    dense FP4 of that residual.
 
     Returns canonical (unpacked, unswizzled) arrays:
       xh [T,K] f32, idx [T,G,n], sp_codes [T,K*n/m] u8, sp_scales [T,nb_sp] u8,
@@ -333,7 +333,7 @@ def prepare_swiglu(gate_up, n: int, m: int, unit: int, fmt: str) -> dict:
 
 
 def quantize_dense(x, gamma, eps: float, fmt: str) -> dict:
-    """The plain dense FP4 activation quantizer (the README's "NVFP4: dense FP4 baseline" mode).
+    """The plain dense FP4 activation quantizer (the README mirror's dense-only NVFP4 mode).
 
     Same row scale and block rule as the residual path, applied to xh itself.
     """
@@ -347,8 +347,8 @@ def quantize_dense(x, gamma, eps: float, fmt: str) -> dict:
 # step a6: the weight payload and its two scale views
 # --------------------------------------------------------------------------------------
 def pack_weight(w, fmt: str, density_den: int = 2) -> dict:
-    """One FP4 weight payload with path-specific scale views (Abstract: "The two
-    paths share a single FP4 weight payload with path-specific scale views").
+    """One FP4 weight payload with path-specific scale views (Abstract: both GEMM
+    paths read the same FP4 weight codes, each with scales laid out for that path).
 
     The weight [N, K] (bf16 values as float32) is quantized once in blocks of
     ``density_den * B`` consecutive K positions, the K span one backbone block
@@ -411,9 +411,9 @@ def dequant_prep(p: dict):
 def linear(p: dict, wp: dict) -> np.ndarray:
     """Y [T, Nout] float64 = A_sp . W_sparse_view^T + A_res . W_dense_view^T.
 
-    Abstract: "A sparse FP4 GEMM processes the backbone while a dense FP4 GEMM
-    compensates for both mask-induced activation loss and sparse-path
-    quantization error." Every dequantized value is exact in float64, so the
+    Abstract: the backbone goes through a sparse FP4 GEMM, the residual through a
+    dense FP4 GEMM that restores what the mask dropped and the backbone's
+    quantization error. Every dequantized value is exact in float64, so the
     only rounding is the float64 sum.
     """
     a_sp, a_res = dequant_prep(p)

@@ -38,16 +38,55 @@ def assert_exact(got, ref):
                                  f"got {a[tuple(bad[0])]} want {b[tuple(bad[0])]}")
 
 
-def assert_close_norm(got, ref):
-    assert np.array_equal(got["idx"], ref["idx"]) or np.mean(got["idx"] != ref["idx"]) <= 1e-4
+_KEYS = ("idx", "sp_codes", "sp_scales", "res_codes", "res_scales", "row_scale")
+
+
+def _row_with_rstd_step(x, gamma, eps, ref, r, step):
+    """The oracle's row r quantized from xh built with rstd moved by `step` float32 ulps.
+
+    Diagnostic only: the GPU and the oracle sum x^2 in float64 in different orders, so
+    fp32(sum/K) -- hence rstd -- may differ by one ulp on rare rows. A differing row is
+    accounted for when it equals the oracle's result under such a neighbouring rstd."""
+    x = np.asarray(x[r:r + 1], np.float32)
+    K = x.shape[1]
+    ss = np.sum(x.astype(np.float64) ** 2, axis=1)
+    rstd = np.float32(1.0) / np.sqrt((ss / np.float64(K)).astype(np.float32) + np.float32(eps))
+    rstd = np.nextafter(rstd, np.float32(np.inf) if step > 0 else np.float32(0))
+    xh = ((x * rstd[:, None]).astype(np.float32) * np.asarray(gamma, np.float32)[None, :]).astype(np.float32)
+    return O.prepare(xh, None, 0.0, ref["n"], ref["m"], ref["unit"], ref["fmt"])
+
+
+def assert_close_norm(got, ref, x=None, gamma=None, eps=None):
+    """Fused-RMSNorm parity: at most 1e-4 of the codes differ, each by one E2M1 step. Mask
+    flips and block-scale flips are counted and bounded on their own (each <= 1e-4 of its
+    entries), and when the inputs are given every row that differs at all must equal the
+    oracle's row under an rstd one float32 ulp away."""
+    counts = {}
     for key in ("sp_codes", "res_codes"):
         diff = got[key] != ref[key]
+        counts[key] = int(diff.sum())
         assert diff.mean() <= 1e-4, (key, diff.mean())
         if diff.any():
             assert code_steps(got[key][diff], ref[key][diff]).max() <= 1
+    counts["mask_flips"] = int((got["idx"] != ref["idx"]).any(axis=2).sum())
+    assert counts["mask_flips"] <= 1e-4 * ref["idx"].shape[0] * ref["idx"].shape[1], counts
     for key in ("sp_scales", "res_scales"):
-        assert np.mean(got[key] != ref[key]) <= 1e-4
+        counts[key] = int((got[key] != ref[key]).sum())
+        assert counts[key] <= 1e-4 * got[key].size, counts
     np.testing.assert_allclose(got["row_scale"], ref["row_scale"], rtol=2 ** -22)
+    rows = sorted({int(r) for key in _KEYS for r in np.argwhere(
+        (got[key] != ref[key]).reshape(got[key].shape[0], -1).any(axis=1)).ravel()})
+    if rows:
+        print(f"fused-RMSNorm rows differing from the oracle: {rows}; counts {counts}")
+    if x is not None:
+        for r in rows:
+            ok = False
+            for step in (-1, 1):
+                alt = _row_with_rstd_step(x, gamma, eps, ref, r, step)
+                if all(np.array_equal(got[k][r:r + 1], alt[k]) for k in _KEYS):
+                    ok = True
+                    break
+            assert ok, f"row {r} differs from the oracle beyond a one-ulp rstd"
 
 
 CASES = [  # (workload, rows) -- tiny: 64x256; ragged: 200 rows (not a multiple of 128)
@@ -74,8 +113,10 @@ def test_prep_bit_exact_without_norm(fmt, unit, name, rows):
 @pytest.mark.parametrize("name,rows", CASES)
 def test_prep_with_fused_rmsnorm(fmt, unit, name, rows):
     S = require_gpu()
-    got, ref = run_prep(S, workload(name), fmt, unit, use_norm=True, rows=rows)
-    assert_close_norm(got, ref)
+    lin = workload(name)
+    got, ref = run_prep(S, lin, fmt, unit, use_norm=True, rows=rows)
+    x = f32(lin.x if rows is None else lin.x[rows])
+    assert_close_norm(got, ref, x, f32(lin.gamma), lin.eps)
 
 
 @pytest.mark.parametrize("fmt", [0, 1])
@@ -112,7 +153,7 @@ def test_prep_edge_values():
             assert_exact(got, ref)
             lin1 = wl.Linear("one", x[4:5], gamma, x)
             got, ref = run_prep(S, lin1, fmt, unit, use_norm=True)
-            assert_close_norm(got, ref)
+            assert_close_norm(got, ref, f32(x[4:5]), f32(gamma), lin1.eps)
 
 
 @pytest.mark.parametrize("fmt", [0, 1])
@@ -148,4 +189,7 @@ def test_prep_full_size_sampled_rows(which, T):
     rows = np.concatenate([rows, [0, T - 1]])
     ref = O.prepare(f32(lin.x[rows]), f32(lin.gamma), lin.eps, 2, 4, 2, O.NVFP4)
     sub = {k: v[rows] for k, v in got.items()}
-    (assert_close_norm if g is not None else assert_exact)(sub, ref)
+    if g is not None:
+        assert_close_norm(sub, ref, f32(lin.x[rows]), f32(lin.gamma), lin.eps)
+    else:
+        assert_exact(sub, ref)

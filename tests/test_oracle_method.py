@@ -281,6 +281,37 @@ def test_linear_matches_triple_loop(fmt, unit):
             assert math.isclose(acc, Y[t, n_], rel_tol=1e-12, abs_tol=1e-12)
 
 
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+def test_linear_dense_matches_triple_loop(fmt):
+    """Brute force for the dense FP4 baseline: every activation code, its block scale and the
+    row scale, every weight code with its dense-view scale and s_w, decoded by library codecs
+    and summed in Python one output at a time (fused RMSNorm on, outlier channels present)."""
+    rng = np.random.default_rng(12)
+    T, K, N = 3, 128, 5
+    x = wl.bf16_bits_to_f32(wl.f32_to_bf16_bits(rng.standard_normal((T, K)).astype(F32) * 3))
+    x[:, 5] *= 60
+    x[1] *= 1e-3                                            # rows with very different scales
+    gamma = wl.bf16_bits_to_f32(wl.f32_to_bf16_bits(rng.uniform(0.5, 1.5, K).astype(F32)))
+    w = wl.bf16_bits_to_f32(wl.f32_to_bf16_bits(rng.standard_normal((N, K)).astype(F32) * 0.02))
+    q = O.quantize_dense(x, gamma, 1e-6, fmt)
+    wp = O.pack_weight(w, fmt)
+    Y = O.linear_dense(q, wp)
+    B = O.block_size(fmt)
+    a_vals = _decode_lib(q["codes"])
+    a_sc = _scale_lib(q["scales"], fmt)
+    w_vals = _decode_lib(wp["codes"])
+    w_sc = _scale_lib(wp["scales_dense"], fmt)
+    s_w = float(wp["tensor_scale"])
+    assert len({float(s) for s in q["row_scale"]}) == (T if fmt == O.NVFP4 else 1)
+    for t in range(T):
+        s_x = float(q["row_scale"][t])
+        for n_ in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc += (a_vals[t, k] * a_sc[t, k // B] * s_x) * (w_vals[n_, k] * w_sc[n_, k // B] * s_w)
+            assert math.isclose(acc, Y[t, n_], rel_tol=1e-12, abs_tol=1e-300)
+
+
 def test_sharq_error_below_dense_nvfp4_on_outlier_inputs():
     """Method sanity: against the bf16 product xh.W^T, SharQ's output error is below dense NVFP4's
     (the abstract's accuracy claim, checked as an inequality on synthetic outlier inputs)."""
