@@ -72,6 +72,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sharq_linear_grouped": (I, [ctypes.POINTER(_Prep), ctypes.POINTER(_WPack), ctypes.POINTER(P), I, I, P]),
         "sharq_quantize_dense": (I, [P, I, I, P, F, I, P, P, P]),
         "sharq_linear_dense": (I, [P, P, I, I, ctypes.POINTER(_WPack), P, I, P]),
+        "sharq_rmsnorm": (I, [P, I, I, P, F, P, P]),
         "sharq_device_status": (I, [P]),
         "sharq_set_wait_limit": (None, [ctypes.c_longlong]),
         "sharq_last_error": (ctypes.c_char_p, []),
@@ -313,6 +314,16 @@ def sharq_linear_dense(q: DenseQ, w: WPack, y: torch.Tensor | None = None, out_d
     _check(lib.sharq_linear_dense(_ptr(q.tiles), _ptr(q.row_scale), q.tokens, q.k, ctypes.byref(w.struct()),
                                   _ptr(y), code, _stream(stream)))
     return y
+
+
+def sharq_rmsnorm(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6, out: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """The dense baseline's separate RMSNorm pass: y = bf16(fp32(fp32(x*rstd)*gamma))."""
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and gamma.dtype == torch.bfloat16
+    tokens, k = x.shape
+    out = torch.empty_like(x) if out is None else out
+    _check(lib.sharq_rmsnorm(_ptr(x), tokens, k, _ptr(gamma), float(eps), _ptr(out), _stream(stream)))
+    return out
 
 
 def sharq_device_status(stream=None) -> int:

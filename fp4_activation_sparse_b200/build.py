@@ -13,7 +13,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsharq.so")
-SOURCES = ["sharq_api.cu", "sharq_prep.cu", "sharq_pack.cu", "sharq_gemm.cu"]
+SOURCES = ["sharq_api.cu", "sharq_prep.cu", "sharq_pack.cu", "sharq_gemm.cu", "sharq_norm.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

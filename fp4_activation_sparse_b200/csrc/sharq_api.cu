@@ -126,6 +126,7 @@ static int prepare_common(const void *x, int tokens, int k, const void *gamma, f
   if (!aligned16(tiles) || !aligned16(row_scale)) return fail(SHARQ_ERR_INVALID_ARG, "output buffers must be 16-byte aligned");
   if (gamma && !(eps >= 0.f)) return fail(SHARQ_ERR_INVALID_ARG, "eps must be >= 0");
   sharq::PrepParams p;
+  memset(&p, 0, sizeof p);
   p.x = static_cast<const uint16_t *>(x);
   p.x_stride = swiglu ? 2 * k : k;
   p.gamma = static_cast<const uint16_t *>(gamma);
@@ -317,6 +318,19 @@ int sharq_linear_dense(const void *tiles, const float *row_scale, int tokens, in
   g.out_f32 = out_dtype == SHARQ_OUT_F32;
   g.sparse = 0;
   return run_gemm(g, "sharq_linear_dense", static_cast<cudaStream_t>(stream));
+}
+
+int sharq_rmsnorm(const void *x, int tokens, int k, const void *gamma, float eps, void *y, void *stream) {
+  if (!x || !gamma || !y) return fail(SHARQ_ERR_INVALID_ARG, "null x, gamma or output");
+  if (int s = check_shape(tokens, k, "tokens")) return s;
+  if (k > 32768) return fail(SHARQ_ERR_INVALID_ARG, "k must be <= 32768 (got %d)", k);
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(y)) return fail(SHARQ_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
+  if (!(eps >= 0.f)) return fail(SHARQ_ERR_INVALID_ARG, "eps must be >= 0");
+  cudaError_t e = sharq::launch_rmsnorm(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(gamma), eps,
+                                        tokens, k, static_cast<uint16_t *>(y), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "sharq_rmsnorm");
+  g_err[0] = 0;
+  return SHARQ_OK;
 }
 
 int sharq_device_status(void *stream) {

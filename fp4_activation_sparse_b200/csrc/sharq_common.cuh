@@ -98,9 +98,43 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t h2) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Correctly rounded 1/d for normal d whose reciprocal is normal: the hardware approximation
+// refined by one fused multiply-add step (P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990: with y faithful to 1/d,
+// the residual e = 1 - d*y is exact and RN(y + y*e) = RN(1/d)). tests/cuda/rcp_check.cu checks
+// it bit for bit against the correctly rounded reciprocal over every such float32.
+__device__ __forceinline__ float rcp_rn(float d) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(d));
+  const float e = __fmaf_rn(-d, y, 1.0f);
+  return __fmaf_rn(y, e, y);
+}
+
+// max(|a|, |b|, |c|) in one instruction
+__device__ __forceinline__ float max3abs(float a, float b, float c) {
+  float d;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // 2^(e-127) as float32 (e in 0..254; e = 0 is the subnormal 2^-127).
 __device__ __forceinline__ float e8m0_to_f32(uint32_t e) {
   return e == 0 ? __uint_as_float(0x00400000u) : __uint_as_float(e << 23);
+}
+
+// Exact squares of a word's two bf16 values added to a float64 sum (low half first), without
+// conversion instructions: the bf16 exponent and mantissa bits of |x|, moved to the top of a
+// float64 high word, encode a = |x| * 2^-896 exactly (zero and subnormal values included);
+// the same bits with 1792 added to the exponent field encode b = |x| * 2^896 for every normal
+// x, so a*b = x^2 exactly (16 significant bits) and zero contributes exactly 0. (A subnormal
+// bf16, |x| < 2^-126, contributes below 2^-252 instead of x^2: far below the float64 rounding
+// of any row sum the contract admits.)
+__device__ __forceinline__ double add_squares_exact(uint32_t w, double ss) {
+  const uint32_t al = (w & 0x7FFFu) << 13, ah = (w >> 3) & 0x0FFFE000u;  // low / high value
+  constexpr uint32_t kUp = 1792u << 20;
+  const double a0 = __hiloint2double((int)al, 0), b0 = __hiloint2double((int)(al + kUp), 0);
+  const double a1 = __hiloint2double((int)ah, 0), b1 = __hiloint2double((int)(ah + kUp), 0);
+  return __fma_rn(a1, b1, __fma_rn(a0, b0, ss));
 }
 
 }  // namespace sharq

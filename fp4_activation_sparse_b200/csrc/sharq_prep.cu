@@ -166,6 +166,14 @@ __device__ __forceinline__ void normalize16(float *v, const float4 *g4, float rs
   }
 }
 
+// max over m and the 16 values |v[i]| (a tree of three-input maxima)
+__device__ __forceinline__ float amax16(const float *v, float m) {
+  const float t0 = max3abs(v[0], v[1], v[2]), t1 = max3abs(v[3], v[4], v[5]), t2 = max3abs(v[6], v[7], v[8]);
+  const float t3 = max3abs(v[9], v[10], v[11]), t4 = max3abs(v[12], v[13], v[14]);
+  const float u0 = max3abs(t0, t1, t2), u1 = max3abs(t3, t4, v[15]);
+  return max3abs(m, u0, u1);
+}
+
 // ---------------------------------------------------------------- block scales
 // NVFP4: E4M3 code of fp32(amax*g); d = fp32(dec*s); inv = 1/d (0 when d = 0).
 struct NvScale {
@@ -180,7 +188,7 @@ __device__ __forceinline__ NvScale nv_scale(float amax, float s_x, float g_x) {
   s.dec = e4m3_to_f32(s.code);
   const float d = __fmul_rn(s.dec, s_x);
   s.zero = d == 0.f;
-  s.inv = s.zero ? 0.f : __frcp_rn(d);
+  s.inv = s.zero ? 0.f : rcp_rn(d);  // d normal: the row-scale contract
   return s;
 }
 
@@ -357,9 +365,7 @@ __device__ __forceinline__ void process16(uint8_t *chunk, const Spot &o, float *
     for (int i = 0; i < 16; i += 2) sub2(v[i], v[i + 1], dq[i], dq[i + 1]);
   }
   // ---- residual (or xh itself for the dense quantizer): dense blocks
-  float am = 0.f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(v[i]));
+  float am = amax16(v, 0.f);
   uint32_t r0, r1, sc_res;
   if (FMT == kFmtNV) {  // block = this lane's 16 values
     const NvScale s = nv_scale(am, s_x, g_x);
@@ -485,8 +491,7 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
       float v[16];
       unpack16(xr[i], v);
       if (NORM) normalize16<true>(v, g_lane + i * 128 * W, rstd);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) am = fmaxf(am, fabsf(v[j]));
+      am = amax16(v, am);
     }
   }
   am = team_max(am, W, team, wt, sm_f);

@@ -209,6 +209,17 @@ int sharq_quantize_dense(const void *x_bf16_dev, int tokens, int k, const void *
 int sharq_linear_dense(const void *tiles_dev, const float *row_scale_dev, int tokens, int k,
                        const sharq_wpack *w, void *y_dev, int out_dtype, void *stream);
 
+/* The separate normalization pass of the dense baseline pipeline (one launch):
+ * y = bf16_RNE(fp32(fp32(x * rstd) * gamma)), rstd = 1/sqrt(fp32(sum(x^2)/k) + eps) with the
+ * sum of squares in float64 -- the value the fused preparation operator normalizes to,
+ * rounded to bf16 as an unfused pipeline passes it to the next kernel. The baseline then runs
+ * sharq_quantize_dense on y without gamma and sharq_linear_dense. The fused preparation
+ * operator replaces this pass (Abstract: normalization folded into the preparation kernel).
+ *   x_bf16_dev, y_bf16_dev  [tokens][k] row-major bf16 (16-byte aligned); k <= 32768
+ *   gamma_bf16_dev          [k] bf16 */
+int sharq_rmsnorm(const void *x_bf16_dev, int tokens, int k, const void *gamma_bf16_dev, float eps,
+                  void *y_bf16_dev, void *stream);
+
 /* Synchronizes `stream`, then reports and clears the device-side status word that
  * bounded waits set when they give up: SHARQ_OK or SHARQ_ERR_TIMEOUT (or SHARQ_ERR_CUDA). */
 int sharq_device_status(void *stream);
