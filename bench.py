@@ -42,6 +42,12 @@ L2_BYTES = 126 * 2 ** 20
 PREP_BYTES_PER_ELEM = 2 + 0.25 + 1 / 16 + 1 / 32 + 0.5 + 1 / 16
 
 
+def prep_bytes_per_elem(fmt: str) -> float:
+    """PREP_BYTES_PER_ELEM for either format (MXFP4: one scale per 32 elements)."""
+    blk = 16 if fmt == "nvfp4" else 32
+    return 2 + 0.25 + 1 / 16 + 0.5 / blk + 0.5 + 1 / blk
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -325,17 +331,43 @@ def run_sharq(args, rank, world, local):
     t_prep_ms = graph_time(prep_graph, nsets)
     t_lin_ms = graph_time(lin_graph, nsets)
 
-    # ---- baselines on the same shapes: torch bf16 matmul and the library's dense NVFP4 pipeline
-    q = S.sharq_quantize_dense(xs[0], gamma, lin.eps, "nvfp4")
-    yd = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
+    # ---- baselines on the same shapes and the same rotating input sets: torch bf16 matmul and
+    # the library's dense NVFP4 pipeline, (a) with the normalization fused into the dense
+    # quantizer and (b) as the separate pipeline SharQ's fused preparation replaces -- an RMSNorm
+    # pass writing bf16, dense quantization of that, the dense FP4 GEMM
     w_bf16 = to_dev(lin.w)
     with torch.cuda.stream(cap):  # cuBLAS creates its handle and workspace outside the capture
         torch.matmul(xs[0], w_bf16.t())
     torch.cuda.synchronize()
-    t_bf16 = graph_time(capture(lambda st: torch.matmul(xs[0], w_bf16.t())), 1)
-    t_dq = graph_time(capture(lambda st: S.sharq_quantize_dense(xs[0], gamma, lin.eps, "nvfp4", out=q, stream=st)), 1)
-    t_dl = graph_time(capture(lambda st: S.sharq_linear_dense(q, wps[0], y=yd, stream=st)), 1)
+    t_bf16 = graph_time(capture(lambda st: [torch.matmul(xs[s], w_bf16.t(), out=ys[s]) for s in range(nsets)]), nsets)
     del w_bf16
+    qs = [S.sharq_quantize_dense(xs[s], gamma, lin.eps, "nvfp4") for s in range(nsets)]
+    xns = [torch.empty_like(xs[0]) for _ in range(nsets)]
+    torch.cuda.synchronize()
+
+    def dense_fused(st):
+        for s in range(nsets):
+            S.sharq_quantize_dense(xs[s], gamma, lin.eps, "nvfp4", out=qs[s], stream=st)
+            S.sharq_linear_dense(qs[s], wps[s], y=ys[s], stream=st)
+
+    def dense_separate(st):
+        for s in range(nsets):
+            S.sharq_rmsnorm(xs[s], gamma, lin.eps, out=xns[s], stream=st)
+            S.sharq_quantize_dense(xns[s], None, 0.0, "nvfp4", out=qs[s], stream=st)
+            S.sharq_linear_dense(qs[s], wps[s], y=ys[s], stream=st)
+
+    t_dense_fused = graph_time(capture(dense_fused), nsets)
+    t_dense_sep = graph_time(capture(dense_separate), nsets)
+    t_norm = graph_time(capture(lambda st: [S.sharq_rmsnorm(xs[s], gamma, lin.eps, out=xns[s], stream=st)
+                                            for s in range(nsets)]), nsets)
+    t_dq = graph_time(capture(lambda st: [S.sharq_quantize_dense(xs[s], gamma, lin.eps, "nvfp4", out=qs[s], stream=st)
+                                          for s in range(nsets)]), nsets)
+    t_dq_plain = graph_time(capture(lambda st: [S.sharq_quantize_dense(xns[s], None, 0.0, "nvfp4", out=qs[s],
+                                                                       stream=st) for s in range(nsets)]), nsets)
+    t_dl = graph_time(capture(lambda st: [S.sharq_linear_dense(qs[s], wps[s], y=ys[s], stream=st)
+                                          for s in range(nsets)]), nsets)
+    t_sharq_step = graph_time(run_graph, nsets)  # SharQ step timed the same way as the pipelines above
+    del qs, xns
 
     # ---- the gated-activation preparation (down projection fed by its gate/up output):
     # fused kernel vs the unfused pipeline (torch SiLU * up in bf16, then the preparation)
@@ -407,6 +439,64 @@ def run_sharq(args, rank, world, local):
                                           for s in range(nsets)]), nsets)
     sw_gbs = sw_bytes / (t_sw / 1e3) / 1e9
     del gus
+
+    # ---- the other configured shapes (Llama-3.1-8B MLP, Qwen2.5-7B linears over M, the 8192^3
+    # square and the video-DiT linear, both formats): prep, linear and whole step, each replayed
+    # as a CUDA graph over enough rotating input sets (activation, weight pack, output) that
+    # every launch reads data last touched more than L2 bytes earlier. Inputs are drawn on the
+    # device with the same recipes.
+    def measure_linear(name, T_, K_, N_, norm, fmt, seed, swiglu_input=False):
+        foot = T_ * K_ * prep_bytes_per_elem(fmt) + N_ * K_ * 0.6 + T_ * N_ * 2
+        n = int(min(32, max(1, np.ceil(3 * L2_BYTES / foot))))
+        x0 = (wl.swiglu_activations_device(seed, T_, K_) if swiglu_input else
+              wl.outlier_activations_device(seed, T_, K_, max(1, K_ // 100), 20.0, 100.0, 0.5))
+        g_ = wl.rms_gamma_device(seed + 1, K_) if norm else None
+        w0 = wl.weight_device(seed + 2, N_, K_)
+        xs_ = [x0] + [x0.clone() for _ in range(n - 1)]
+        wps_ = [S.sharq_pack_weight(w0, fmt) for _ in range(n)]
+        del w0
+        ps = [S.alloc_prep(T_, K_, 2, 4, 2, fmt) for _ in range(n)]
+        ys_ = [torch.empty(T_, N_, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+
+        def prep_all(st):
+            for i in range(n):
+                S.sharq_prepare(xs_[i], g_, 1e-6, 2, 4, 2, fmt, out=ps[i], stream=st)
+
+        def lin_all(st):
+            for i in range(n):
+                S.sharq_linear(ps[i], wps_[i], y=ys_[i], stream=st)
+
+        def step_all(st):
+            for i in range(n):
+                S.sharq_prepare(xs_[i], g_, 1e-6, 2, 4, 2, fmt, out=ps[i], stream=st)
+                S.sharq_linear(ps[i], wps_[i], y=ys_[i], stream=st)
+
+        step_all(stream)
+        torch.cuda.synchronize()
+        tp, tl, ts = (graph_time(capture(f), n) for f in (prep_all, lin_all, step_all))
+        pb = T_ * K_ * prep_bytes_per_elem(fmt) + T_ * 4 + (K_ * 2 if norm else 0)
+        gt = 3.0 * T_ * N_ * K_ / (tl / 1e3) / 1e12
+        return {"workload": name, "T": T_, "K": K_, "N": N_, "fmt": fmt, "fused_rmsnorm": norm,
+                "t_prep_us": tp * 1e3, "t_linear_us": tl * 1e3, "t_step_us": ts * 1e3,
+                "tokens_per_s": T_ / (ts / 1e3), "eff_fp4_tflops": 2.0 * T_ * N_ * K_ / (ts / 1e3) / 1e12,
+                "gemm_tflops": gt, "gemm_frac": gt / fp4_dense_peak,
+                "prep_gbs": pb / (tp / 1e3) / 1e9, "prep_frac": pb / (tp / 1e3) / 1e9 / hbm_peak,
+                "l2": f"{n} rotating set(s)"}
+
+    sweep = []
+    if not args.no_sweep:
+        cases = [("llama31_8b_qkv_prefill", 16384, 4096, 6144, True, "nvfp4", False),
+                 ("llama31_8b_gate_up", 4096, 4096, 28672, True, "nvfp4", False),
+                 ("llama31_8b_down", 4096, 14336, 4096, False, "nvfp4", True)]
+        for which, (Kq, Nq, normq) in wl.QWEN_LINEARS.items():
+            for Tq in (1, 16, 128, 2048, 8192):
+                cases.append((f"qwen25_7b_{which}", Tq, Kq, Nq, normq, "nvfp4", False))
+        for fmt_ in ("nvfp4", "mxfp4"):
+            cases.append(("square_8192", 8192, 8192, 8192, False, fmt_, False))
+            cases.append(("video_dit", 32760, 5120, 5120, False, fmt_, False))
+        for ci, c in enumerate(cases):
+            sweep.append(measure_linear(*c[:6], seed=9000 + 10 * ci, swiglu_input=c[6]))
+        assert S.sharq_device_status() == S.SHARQ_OK
 
     # ---- end to end through the public API with host buffers: every step copies its input
     # from pinned host memory and its output back. Copies run on their own streams and overlap
@@ -486,8 +576,15 @@ def run_sharq(args, rank, world, local):
         "t_prep_us": t_prep_ms * 1e3, "t_linear_us": t_lin_ms * 1e3,
         "roofline": dominant, "roofline_prep": rf_prep, "roofline_gemm": rf_gemm,
         "baselines": {"torch_bf16_matmul_us": t_bf16 * 1e3,
-                      "dense_nvfp4_pipeline_us": (t_dq + t_dl) * 1e3,
-                      "dense_nvfp4_quantize_us": t_dq * 1e3, "dense_nvfp4_gemm_us": t_dl * 1e3},
+                      "sharq_step_us": t_sharq_step * 1e3,
+                      "dense_nvfp4_separate_prep_pipeline_us": t_dense_sep * 1e3,
+                      "dense_nvfp4_fused_quantizer_pipeline_us": t_dense_fused * 1e3,
+                      "sharq_vs_dense_nvfp4": t_dense_sep / t_sharq_step,
+                      "sharq_vs_dense_nvfp4_fused_quantizer": t_dense_fused / t_sharq_step,
+                      "rmsnorm_us": t_norm * 1e3, "dense_nvfp4_quantize_us": t_dq_plain * 1e3,
+                      "dense_nvfp4_quantize_with_norm_us": t_dq * 1e3, "dense_nvfp4_gemm_us": t_dl * 1e3,
+                      "note": "pipelines and the SharQ step each replayed as one CUDA graph over the same rotating "
+                              "input sets; ratios are dense time / SharQ time (> 1: SharQ faster)"},
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * K * 2,
                 "d2h_bytes_per_step": T * N * 2},
         "next": {"swiglu_prep": {
@@ -498,7 +595,8 @@ def run_sharq(args, rank, world, local):
                 "workload": f"llama31_8b_qkv_prefill T={T} K={K} nvfp4 2:4-pairs fused-rmsnorm, one scale per tensor",
                 "t_us": t_ts * 1e3, "per_row_scale_prep_us": t_prep_ms * 1e3,
                 "note": "3 launches + 4-byte clear; the amax pass reads x a second time"},
-            "moe_grouped": moe_line},
+            "moe_grouped": moe_line,
+            "shapes": sweep},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "device_status": status,
@@ -542,6 +640,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sharq", "reference"], default="sharq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the other configured shapes")
     ap.add_argument("--profile", choices=["prep", "linear", "dense"], help="run 3 launches of one kernel for ncu")
     ap.add_argument("--tokens", type=int, default=2048)
     args = ap.parse_args()

@@ -170,3 +170,42 @@ QWEN3_MOE = dict(hidden=2048, moe_intermediate=768, n_experts=128, top_k=8)  # Q
 def crafted_row(values) -> np.ndarray:
     """bf16 bits of a hand-written row (for edge-case tests)."""
     return f32_to_bf16_bits(np.asarray(values, dtype=np.float32)[None, :])
+
+
+def outlier_activations_device(seed: int, T: int, K: int, n_outlier: int, scale_lo: float, scale_hi: float,
+                               token_sigma: float, device="cuda"):
+    """The recipe of ``outlier_activations`` drawn on the device with torch's generator, for
+    benchmark sizes whose host-side drawing would dominate the run (bf16 tensor [T, K]; the
+    same distribution, not the same bits as the numpy stream)."""
+    import torch
+    g = torch.Generator(device=device).manual_seed(seed)
+    z = torch.randn(T, K, generator=g, device=device)
+    ch = torch.ones(K, device=device)
+    idx = torch.randperm(K, generator=g, device=device)[:n_outlier]
+    ch[idx] = torch.empty(n_outlier, device=device).uniform_(scale_lo, scale_hi, generator=g)
+    tok = torch.ones(T, device=device)
+    if token_sigma > 0:
+        tok = torch.exp(torch.randn(T, generator=g, device=device) * token_sigma)
+    return (z * tok[:, None] * ch[None, :]).to(torch.bfloat16)
+
+
+def swiglu_activations_device(seed: int, T: int, K: int, device="cuda"):
+    """The recipe of ``swiglu_activations`` drawn on the device (bf16 tensor [T, K])."""
+    import torch
+    g = torch.Generator(device=device).manual_seed(seed)
+    a = torch.randn(T, K, generator=g, device=device)
+    u = torch.randn(T, K, generator=g, device=device)
+    return (a / (1.0 + torch.exp(-a)) * u).to(torch.bfloat16)
+
+
+def weight_device(seed: int, N: int, K: int, device="cuda"):
+    """The recipe of ``weight`` drawn on the device (bf16 tensor [N, K], N(0, 0.02))."""
+    import torch
+    g = torch.Generator(device=device).manual_seed(seed)
+    return (torch.randn(N, K, generator=g, device=device) * 0.02).to(torch.bfloat16)
+
+
+def rms_gamma_device(seed: int, K: int, device="cuda"):
+    import torch
+    g = torch.Generator(device=device).manual_seed(seed)
+    return (torch.rand(K, generator=g, device=device) + 0.5).to(torch.bfloat16)
