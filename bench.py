@@ -113,6 +113,43 @@ class ClockSampler:
 CSRC = os.path.join(ROOT, "fp4_activation_sparse_b200", "csrc")
 
 
+def measure_mma_peaks(S, local: int, stream) -> dict:
+    """Tensor-core ceilings from the library's peak loop (sharq_mma_peak: the GEMM's own MMAs,
+    resident operands, one CTA pair per SM pair), both formats and modes. Burst: one launch of
+    about 3 ms per mode after a short idle pause (the GEMM's own timings are bursts of a few
+    ms); sustained: the SharQ K step for about 1 s, where the power cap lowers the clock.
+    Rates of mode 2 are in the GEMM's dense-equivalent units."""
+    pairs = torch.cuda.get_device_properties(local).multi_processor_count // 2
+    names = {0: "dense", 1: "sparse_logical", 2: "sharq_step"}
+
+    def rate(mode, fmt, iters, reps):
+        S.sharq_mma_peak(mode, fmt, 256, stream=stream)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            S.sharq_mma_peak(mode, fmt, iters, stream=stream)
+        b.record(stream)
+        b.synchronize()
+        return S.MMA_PEAK_STEP_FLOPS[mode] * iters * reps * pairs / (a.elapsed_time(b) / 1e3) / 1e12
+
+    out = {"burst": {}, "sustained": {}}
+    with ClockSampler(local) as clk_b:
+        for fmt in ("nvfp4", "mxfp4"):
+            for mode in (0, 1, 2):
+                time.sleep(0.2)
+                out["burst"][f"{fmt}_{names[mode]}_tflops"] = rate(mode, fmt, 8192, 1)
+    with ClockSampler(local) as clk_s:
+        for fmt in ("nvfp4", "mxfp4"):
+            out["sustained"][f"{fmt}_sharq_step_tflops"] = rate(2, fmt, 65536, 8)
+    assert S.sharq_device_status() == S.SHARQ_OK
+    out["burst"]["clocks"] = clk_b.summary()
+    out["sustained"]["clocks"] = clk_s.summary()
+    out["how"] = (f"sharq_mma_peak: {pairs} CTA pairs, each K step M=256 x N=256 x 256 K of the GEMM's MMAs from "
+                  "resident shared and tensor memory; burst 8192 steps (1 launch per mode, 0.2 s pause before "
+                  "each), sustained 8 x 65536 steps; CUDA events")
+    return out
+
+
 def profiled_traffic(profile: str, sources: list[str], rows: int) -> float | None:
     """DRAM bytes (read + write) per launch from a committed ncu summary under profiles/, or
     None when the kernel's sources changed since the capture (hash recorded in the summary)."""
@@ -241,7 +278,6 @@ def run_reference(args, rank, world):
 def run_sharq(args, rank, world, local):
     import fp4_activation_sparse_b200 as S
     hbm_peak, bf16_peak, bf16_sust, peak_src = load_peaks()
-    fp4_dense_peak = bf16_peak * 4.0  # nominal FP4:BF16 dense ratio 9 : 2.25 applied to the measured bf16 peak
 
     lin = wl.llama_qkv(T=2048, seed=replica_seed(rank))
     T, K, N = lin.shape
@@ -330,6 +366,12 @@ def run_sharq(args, rank, world, local):
 
     t_prep_ms = graph_time(prep_graph, nsets)
     t_lin_ms = graph_time(lin_graph, nsets)
+
+    # ---- tensor-core ceilings of the GEMM's instruction mix, measured now on this GPU
+    mma_peaks = measure_mma_peaks(S, local, stream)
+    fp4_peak = {f: mma_peaks["burst"][f"{f}_sharq_step_tflops"] for f in ("nvfp4", "mxfp4")}
+    fp4_peak_src = ("measured (burst): sharq_mma_peak mode 2, the GEMM's K-step MMA mix from resident operands, "
+                    f"median SM clock {mma_peaks['burst']['clocks'].get('sm_mhz')} MHz")
 
     # ---- baselines on the same shapes and the same rotating input sets: torch bf16 matmul and
     # the library's dense NVFP4 pipeline, (a) with the normalization fused into the dense
@@ -429,7 +471,8 @@ def run_sharq(args, rank, world, local):
     moe_line = {"workload": f"qwen3_30b_a3b experts gate_up T={T} top-{moe['top_k']} of {E}, K={Km} N={Nm} nvfp4",
                 "routed_rows": int(counts.sum()), "padded_rows": rows_pad, "launches": "1 prep + "
                 f"{(E + 31) // 32} grouped GEMM", "t_prep_us": t_moe_prep * 1e3, "t_grouped_gemm_us": t_moe_gemm * 1e3,
-                "achieved_tflops": moe_tflops, "peak_tflops": fp4_dense_peak, "frac": moe_tflops / fp4_dense_peak}
+                "achieved_tflops": moe_tflops, "peak_tflops": fp4_peak["nvfp4"],
+                "frac": moe_tflops / fp4_peak["nvfp4"]}
     del x_moe, x_moe_tok, wps_moe, p_moe, views, ys_moe
 
     # ---- one NVFP4 second-level scale per tensor (amax pass + preparation + scale fill)
@@ -479,7 +522,7 @@ def run_sharq(args, rank, world, local):
         return {"workload": name, "T": T_, "K": K_, "N": N_, "fmt": fmt, "fused_rmsnorm": norm,
                 "t_prep_us": tp * 1e3, "t_linear_us": tl * 1e3, "t_step_us": ts * 1e3,
                 "tokens_per_s": T_ / (ts / 1e3), "eff_fp4_tflops": 2.0 * T_ * N_ * K_ / (ts / 1e3) / 1e12,
-                "gemm_tflops": gt, "gemm_frac": gt / fp4_dense_peak,
+                "gemm_tflops": gt, "gemm_frac": gt / fp4_peak[fmt],
                 "prep_gbs": pb / (tp / 1e3) / 1e9, "prep_frac": pb / (tp / 1e3) / 1e9 / hbm_peak,
                 "l2": f"{n} rotating set(s)"}
 
@@ -557,10 +600,10 @@ def run_sharq(args, rank, world, local):
     rf_prep = {"bound": "hbm", "achieved": prep_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": prep_gbs / hbm_peak,
                "traffic": profiled_traffic("prep_kernel_llama_qkv_T16384.md", ["sharq_prep.cu"] + common, T),
                "kernel": "sharq_prep", "peak_source": peak_src}
-    rf_gemm = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_dense_peak, "unit": "TFLOP/s",
-               "frac": gemm_tflops / fp4_dense_peak,
+    rf_gemm = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak["nvfp4"], "unit": "TFLOP/s",
+               "frac": gemm_tflops / fp4_peak["nvfp4"],
                "traffic": profiled_traffic("sharq_gemm_llama_qkv_T2048.md", ["sharq_gemm.cu"] + common, T),
-               "kernel": "sharq_gemm", "peak_source": f"{peak_src} bf16 x 4 (nominal dense FP4:BF16)"}
+               "kernel": "sharq_gemm", "peak_source": fp4_peak_src}
     dominant = rf_gemm if t_lin_ms >= t_prep_ms else rf_prep
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -597,6 +640,7 @@ def run_sharq(args, rank, world, local):
                 "note": "3 launches + 4-byte clear; the amax pass reads x a second time"},
             "moe_grouped": moe_line,
             "shapes": sweep},
+        "mma_peaks": mma_peaks,
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "device_status": status,

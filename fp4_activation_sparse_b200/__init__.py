@@ -73,6 +73,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sharq_quantize_dense": (I, [P, I, I, P, F, I, P, P, P]),
         "sharq_linear_dense": (I, [P, P, I, I, ctypes.POINTER(_WPack), P, I, P]),
         "sharq_rmsnorm": (I, [P, I, I, P, F, P, P]),
+        "sharq_mma_peak": (I, [I, I, I, I, P]),
         "sharq_device_status": (I, [P]),
         "sharq_set_wait_limit": (None, [ctypes.c_longlong]),
         "sharq_last_error": (ctypes.c_char_p, []),
@@ -324,6 +325,17 @@ def sharq_rmsnorm(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6, out: 
     out = torch.empty_like(x) if out is None else out
     _check(lib.sharq_rmsnorm(_ptr(x), tokens, k, _ptr(gamma), float(eps), _ptr(out), _stream(stream)))
     return out
+
+
+# flops one K step of one CTA pair performs in sharq_mma_peak, per mode: dense; sparse (logical,
+# counting the dropped half as NVIDIA's sparse peaks do); both, in sharq_linear's dense-equivalent
+# units (3 * 256^3: the dense path over all of K plus the sparse path over its kept half)
+MMA_PEAK_STEP_FLOPS = {0: 2.0 * 256 ** 3, 1: 2.0 * 256 ** 3, 2: 3.0 * 256 ** 3}
+
+
+def sharq_mma_peak(mode: int, fmt="nvfp4", iters: int = 65536, clusters: int = 0, stream=None) -> None:
+    """Launch the tensor-core peak loop (mode 0 dense, 1 sparse, 2 both); the caller times it."""
+    _check(lib.sharq_mma_peak(int(mode), _fmt(fmt), int(iters), int(clusters), _stream(stream)))
 
 
 def sharq_device_status(stream=None) -> int:

@@ -333,6 +333,17 @@ int sharq_rmsnorm(const void *x, int tokens, int k, const void *gamma, float eps
   return SHARQ_OK;
 }
 
+int sharq_mma_peak(int mode, int fmt, int iters, int clusters, void *stream) {
+  if (mode < 0 || mode > 2) return fail(SHARQ_ERR_INVALID_ARG, "mode must be 0 (dense), 1 (sparse) or 2 (both)");
+  if (!valid_fmt(fmt)) return fail(SHARQ_ERR_INVALID_ARG, "bad fmt %d", fmt);
+  if (iters < 1 || iters > (1 << 20)) return fail(SHARQ_ERR_INVALID_ARG, "iters must be in [1, 2^20] (got %d)", iters);
+  if (clusters < 0) return fail(SHARQ_ERR_INVALID_ARG, "clusters must be >= 0");
+  cudaError_t e = sharq::launch_mma_peak(mode, fmt, iters, clusters, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "sharq_mma_peak");
+  g_err[0] = 0;
+  return SHARQ_OK;
+}
+
 int sharq_device_status(void *stream) {
   int st = 0;
   cudaError_t e = sharq::read_and_clear_device_status(&st, static_cast<cudaStream_t>(stream));

@@ -713,6 +713,154 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
+// ---------------------------------------------------------------- tensor-core peak loop
+// The MMAs of one K step of the kernel above, issued back to back against one shared-memory
+// stage and one tensor-memory scale buffer that stay resident: no loads, no scale writes, no
+// epilogue. A launch on every SM pair measures the rate of the tensor pipe for this exact
+// instruction mix, the ceiling the GEMM is compared with. MODE 0: the four dense MMAs of a K
+// step; 1: the two sparse MMAs; 2: both (the SharQ K step). Operands are pseudo-random E2M1
+// codes (every nibble is a value), block scales in [1/4, 4] and metadata of valid ascending
+// pair indices; the accumulator restarts every 16 K steps, as the GEMM's does at K = 4096.
+constexpr int kPeakThreads = 128;
+constexpr int kPeakSmemBytes = kMaxStageBytes + 64 + 1024;
+
+__device__ __forceinline__ uint32_t hash32(uint32_t x) {  // integer finalizer (xorshift-multiply)
+  x ^= x >> 16;
+  x *= 0x7feb352du;
+  x ^= x >> 15;
+  x *= 0x846ca68bu;
+  x ^= x >> 16;
+  return x;
+}
+
+template <bool MX, int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPeakThreads, 1)
+    mma_peak_kernel(int iters, unsigned long long limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kMaxStageBytes);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 1);
+  using L = Stage<MX, true>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const uint32_t smem0 = smem_u32(smem), done = smem_u32(bars);
+
+  for (int i = threadIdx.x; i < L::kBytes / 4; i += blockDim.x)
+    reinterpret_cast<uint32_t *>(smem)[i] = hash32((uint32_t)i * 2654435761u + rank);
+  if (threadIdx.x == 0) {
+    mbar_init(done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  fence_proxy_async();  // the MMAs read the operands through the async proxy
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  {
+    // scale buffer 0 (columns 256..335) of this warp's lane quarter: metadata in the first 4
+    // columns, scale bytes in the rest
+    const uint32_t base = tmem + ((uint32_t)(warp * 32) << 16) + kAccCols;
+    // valid (i0 < i1) nibbles i0 | i1 << 2: 4 8 C 9 D E, two of them twice, packed 4 bits each
+    constexpr uint32_t kMetaNibbles = 0xE4ED9C84u;
+#pragma unroll 1
+    for (int c = 0; c < (int)kScaleBufCols; c += 16) {
+      uint32_t r[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t h = hash32((uint32_t)((warp * 32 + lane) * kScaleBufCols + c + j) ^ (rank << 20));
+        uint32_t w = 0u;
+        if (c + j < 4) {
+#pragma unroll
+          for (int n = 0; n < 8; ++n) w |= ((kMetaNibbles >> (4 * ((h >> (3 * n)) & 7u))) & 0xFu) << (4 * n);
+        } else {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const uint32_t hb = h >> (8 * b);
+            const uint32_t code = MX ? 125u + (hb & 3u) + ((hb >> 2) & 1u) : ((5u + (hb & 3u)) << 3) | ((hb >> 2) & 7u);
+            w |= code << (8 * b);
+          }
+        }
+        r[j] = w;
+      }
+      tmem_st<16>(base + c, r);
+    }
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (rank == 0 && warp == 1 && lane == 0) {
+    const uint32_t st4 = smem0 >> 4;
+    const uint32_t sbuf = tmem + kAccCols;
+    const uint32_t t_meta = sbuf, t_sfa_sp = sbuf + 4, t_sfa_res = sbuf + 12, t_sfb_sp = sbuf + 28,
+                   t_sfb_res = sbuf + 44;
+    constexpr int kA = 0, kW = L::kW;
+    for (int it = 0; it < iters; ++it) {
+      uint32_t accumulate = (it & 15) ? 1u : 0u;
+      if (MODE != 0) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint32_t atom = MX ? (uint32_t)(j >> 1) : (uint32_t)j;
+          const uint32_t id = MX ? (uint32_t)(2 * (j & 1)) : 0u;
+          mma_sparse<MX>(tmem, dsc(kDescSw64, st4 + (kA + L::A.sp + 32 * j) / 16),
+                         dsc(kDescSw128, st4 + (kW + L::W.b + 64 * j) / 16), t_meta + 2 * j,
+                         idesc_bs(true, MX, id, id), (t_sfa_sp + 4 * atom) | (id << 30),
+                         (t_sfb_sp + 8 * atom) | (id << 30), accumulate);
+          accumulate = 1u;
+        }
+      }
+      if (MODE != 1) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t atom = MX ? (uint32_t)(j >> 1) : (uint32_t)j;
+          const uint32_t id = MX ? (uint32_t)(2 * (j & 1)) : 0u;
+          mma_dense<MX>(tmem, dsc(kDescSw128, st4 + (kA + L::A.res + 32 * j) / 16),
+                        dsc(kDescSw128, st4 + (kW + L::W.b + 32 * j) / 16), idesc_bs(false, MX, id, id),
+                        (t_sfa_res + 4 * atom) | (id << 30), (t_sfb_res + 8 * atom) | (id << 30), accumulate);
+          accumulate = 1u;
+        }
+      }
+    }
+    tc_commit_both(done);  // arrives in both CTAs once every MMA above has completed
+  }
+  if (threadIdx.x == 0) {
+    volatile uint32_t no_abort = 0;
+    mbar_wait(done, 0, limit_ns, &no_abort);  // on expiry the device status records it
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+}
+
+template <bool MX, int MODE>
+cudaError_t launch_peak_t(int iters, int clusters, cudaStream_t st) {
+  static std::once_flag once[64];
+  static cudaError_t err[64];
+  static int sms[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [dev] {
+    err[dev] = cudaFuncSetAttribute(mma_peak_kernel<MX, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kPeakSmemBytes);
+    if (err[dev] == cudaSuccess) err[dev] = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+  });
+  if (err[dev] != cudaSuccess) return err[dev];
+  const int pairs = clusters > 0 && clusters < sms[dev] / 2 ? clusters : sms[dev] / 2;
+  // a wait limit far above the loop's length (~0.5 us per K step at the lowest clocks seen)
+  const unsigned long long limit = 4000000000ull + 2000ull * (unsigned long long)iters;
+  mma_peak_kernel<MX, MODE><<<2 * pairs, kPeakThreads, kPeakSmemBytes, st>>>(iters, limit);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -866,6 +1014,13 @@ cudaError_t launch_gemm(GemmParams p, cudaStream_t st, const char **why) {
   }
   p.num_tiles = tiles;
   return p.n_groups == 1 ? launch_groups<1>(p, st, why) : launch_groups<kMaxGroups>(p, st, why);
+}
+
+cudaError_t launch_mma_peak(int mode, int fmt, int iters, int clusters, cudaStream_t st) {
+  const bool mx = fmt == kFmtMX;
+  if (mode == 0) return mx ? launch_peak_t<true, 0>(iters, clusters, st) : launch_peak_t<false, 0>(iters, clusters, st);
+  if (mode == 1) return mx ? launch_peak_t<true, 1>(iters, clusters, st) : launch_peak_t<false, 1>(iters, clusters, st);
+  return mx ? launch_peak_t<true, 2>(iters, clusters, st) : launch_peak_t<false, 2>(iters, clusters, st);
 }
 
 cudaError_t read_and_clear_device_status(int *status, cudaStream_t st) {

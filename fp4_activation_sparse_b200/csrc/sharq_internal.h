@@ -89,6 +89,7 @@ cudaError_t launch_prep_tensor_scale(PrepParams p, int unit, bool norm, cudaStre
 cudaError_t launch_pack(PackParams p, int fmt, cudaStream_t st);
 cudaError_t launch_gemm(GemmParams p, cudaStream_t st, const char **why);
 cudaError_t read_and_clear_device_status(int *status, cudaStream_t st);
+cudaError_t launch_mma_peak(int mode, int fmt, int iters, int clusters, cudaStream_t st);
 cudaError_t launch_rmsnorm(const uint16_t *x, const uint16_t *gamma, float eps, int T, int K, uint16_t *y,
                            cudaStream_t st);
 

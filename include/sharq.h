@@ -220,6 +220,21 @@ int sharq_linear_dense(const void *tiles_dev, const float *row_scale_dev, int to
 int sharq_rmsnorm(const void *x_bf16_dev, int tokens, int k, const void *gamma_bf16_dev, float eps,
                   void *y_bf16_dev, void *stream);
 
+/* Diagnostic: the tensor-core ceiling that sharq_linear is measured against. The pages have no
+ * counterpart; this is the measured denominator of the GEMM's tensor-pipe fraction. One
+ * launch, one CTA pair per SM pair (or `clusters` pairs if 0 < clusters < SMs/2), each issuing
+ * `iters` K steps of sharq_linear's MMAs (M = 256 rows over the pair, N = 256, 256 logical K
+ * per step) from one resident shared-memory stage and one tensor-memory scale buffer, with no
+ * loads, scale writes or epilogue. The caller times the launch (CUDA events on `stream`).
+ *   mode   0: the four dense block-scaled MMAs of a K step (2*256*256*256 flops per step);
+ *          1: the two structured-sparse MMAs (2*256*256*256 logical flops, half of them on
+ *             kept values); 2: both, sharq_linear's K step
+ *   fmt    SHARQ_NVFP4 (kind::mxf4nvf4, 16-element E4M3 scales) or SHARQ_MXFP4 (kind::mxf4)
+ *   iters  1 .. 2^20 K steps per pair
+ * Operands are pseudo-random; results are discarded. A completion wait that gives up is
+ * reported by sharq_device_status. */
+int sharq_mma_peak(int mode, int fmt, int iters, int clusters, void *stream);
+
 /* Synchronizes `stream`, then reports and clears the device-side status word that
  * bounded waits set when they give up: SHARQ_OK or SHARQ_ERR_TIMEOUT (or SHARQ_ERR_CUDA). */
 int sharq_device_status(void *stream);
