@@ -67,7 +67,8 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sharq_pack_weight": (I, [P, I, I, I, ctypes.POINTER(_WPack), P]),
         "sharq_prepare": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P]),
         "sharq_prepare_swiglu": (I, [P, I, I, I, I, I, I, ctypes.POINTER(_Prep), P]),
-        "sharq_prepare_tensor_scale": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P]),
+        "sharq_tensor_scale_workspace_size": (S, [I, I]),
+        "sharq_prepare_tensor_scale": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P, P]),
         "sharq_linear": (I, [ctypes.POINTER(_Prep), ctypes.POINTER(_WPack), P, I, P]),
         "sharq_linear_grouped": (I, [ctypes.POINTER(_Prep), ctypes.POINTER(_WPack), ctypes.POINTER(P), I, I, P]),
         "sharq_quantize_dense": (I, [P, I, I, P, F, I, P, P, P]),
@@ -225,19 +226,30 @@ def sharq_prepare(x: torch.Tensor, gamma: torch.Tensor | None = None, eps: float
     return out
 
 
+def sharq_tensor_scale_workspace_size(tokens: int, k: int) -> int:
+    n = lib.sharq_tensor_scale_workspace_size(tokens, k)
+    if n == 0:
+        raise SharqError(SHARQ_ERR_INVALID_ARG, last_error())
+    return n
+
+
 def sharq_prepare_tensor_scale(x: torch.Tensor, gamma: torch.Tensor | None = None, eps: float = 1e-6,
                                nm_n: int = 2, nm_m: int = 4, unit: int = UNIT_PAIR, fmt="nvfp4",
-                               out: Prep | None = None, stream=None) -> Prep:
+                               out: Prep | None = None, workspace: torch.Tensor | None = None,
+                               stream=None) -> Prep:
     """sharq_prepare with one NVFP4 second-level scale for the whole tensor (every row_scale
-    entry holds it)."""
+    entry holds it). One cooperative launch; `workspace` carries its grid barrier: device bytes
+    zeroed once before first use (allocated zeroed here if omitted), reusable afterwards."""
     assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous()
     tokens, k = x.shape
     if gamma is not None:
         assert gamma.dtype == torch.bfloat16 and gamma.is_cuda and gamma.numel() == k
     out = out or alloc_prep(tokens, k, nm_n, nm_m, unit, fmt, x.device)
+    if workspace is None:
+        workspace = torch.zeros(sharq_tensor_scale_workspace_size(tokens, k), dtype=torch.uint8, device=x.device)
     st = out.struct()
     _check(lib.sharq_prepare_tensor_scale(_ptr(x), tokens, k, _ptr(gamma), ctypes.c_float(eps), nm_n, nm_m, unit,
-                                          _fmt(fmt), ctypes.byref(st), _stream(stream)))
+                                          _fmt(fmt), ctypes.byref(st), _ptr(workspace), _stream(stream)))
     return out
 
 
@@ -344,5 +356,5 @@ def sharq_device_status(stream=None) -> int:
 
 
 def sharq_set_wait_limit(nanoseconds: int) -> None:
-    """Test hook: time limit of the GEMM's bounded waits (0 restores the default of 4 s)."""
+    """Test hook: time limit of the library's bounded device waits (0 restores the default of 4 s)."""
     lib.sharq_set_wait_limit(int(nanoseconds))

@@ -115,7 +115,7 @@ int sharq_pack_weight(const void *w, int n_out, int k, int fmt, sharq_wpack *out
 
 static int prepare_common(const void *x, int tokens, int k, const void *gamma, float eps, int fmt, bool dense,
                           int unit, uint8_t *tiles, float *row_scale, cudaStream_t st, bool swiglu = false,
-                          bool per_tensor = false) {
+                          bool per_tensor = false, void *workspace = nullptr) {
   if (!x) return fail(SHARQ_ERR_INVALID_ARG, "x is null");
   if (!valid_fmt(fmt)) return fail(SHARQ_ERR_INVALID_ARG, "unknown fmt %d", fmt);
   if (int s = check_shape(tokens, k, "tokens")) return s;
@@ -136,8 +136,11 @@ static int prepare_common(const void *x, int tokens, int k, const void *gamma, f
   p.T_pad = sharq::round_up(tokens, 256);
   p.tiles = tiles;
   p.row_scale = row_scale;
-  cudaError_t e = per_tensor && fmt == SHARQ_NVFP4 ? sharq::launch_prep_tensor_scale(p, unit, gamma != nullptr, st)
-                                                   : sharq::launch_prep(p, fmt, unit, gamma != nullptr, dense, swiglu, st);
+  const long long lim = g_wait_limit.load(std::memory_order_relaxed);
+  cudaError_t e = per_tensor && fmt == SHARQ_NVFP4
+                      ? sharq::launch_prep_tensor_scale(p, unit, gamma != nullptr, workspace,
+                                                        lim > 0 ? (unsigned long long)lim : 4000000000ull, st)
+                      : sharq::launch_prep(p, fmt, unit, gamma != nullptr, dense, swiglu, st);
   if (e != cudaSuccess)
     return cuda_fail(e, dense ? "sharq_quantize_dense" : swiglu ? "sharq_prepare_swiglu" : "sharq_prepare");
   g_err[0] = 0;
@@ -161,12 +164,20 @@ int sharq_prepare(const void *x, int tokens, int k, const void *gamma, float eps
   return s;
 }
 
+size_t sharq_tensor_scale_workspace_size(int tokens, int k) {
+  if (check_shape(tokens, k, "tokens")) return 0;
+  if (k > 32768) { fail(SHARQ_ERR_INVALID_ARG, "k must be <= 32768 (got %d)", k); return 0; }
+  return 16 + 4 * (size_t)sharq::prep_tensor_groups(tokens, k);
+}
+
 int sharq_prepare_tensor_scale(const void *x, int tokens, int k, const void *gamma, float eps, int nm_n, int nm_m,
-                               int unit, int fmt, sharq_prep *out, void *stream) {
+                               int unit, int fmt, sharq_prep *out, void *workspace, void *stream) {
   if (!out) return fail(SHARQ_ERR_INVALID_ARG, "output struct is null");
   if (int s = check_pattern(nm_n, nm_m, unit)) return s;
+  if (fmt == SHARQ_NVFP4 && (!workspace || !aligned16(workspace)))
+    return fail(SHARQ_ERR_INVALID_ARG, "workspace must be a 16-byte aligned device buffer");
   int s = prepare_common(x, tokens, k, gamma, eps, fmt, false, unit, static_cast<uint8_t *>(out->tiles),
-                         out->row_scale, static_cast<cudaStream_t>(stream), false, true);
+                         out->row_scale, static_cast<cudaStream_t>(stream), false, true, workspace);
   if (s == SHARQ_OK) {
     out->tokens = tokens;
     out->k = k;
@@ -346,8 +357,11 @@ int sharq_mma_peak(int mode, int fmt, int iters, int clusters, void *stream) {
 
 int sharq_device_status(void *stream) {
   int st = 0;
+  uint32_t prep_st = 0;
   cudaError_t e = sharq::read_and_clear_device_status(&st, static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) e = sharq::read_and_clear_prep_status(&prep_st);
   if (e != cudaSuccess) return cuda_fail(e, "sharq_device_status");
+  st |= (int)(prep_st << 1);
   if (st) return fail(SHARQ_ERR_TIMEOUT, "a bounded device wait gave up (code 0x%x)", st);
   g_err[0] = 0;
   return SHARQ_OK;

@@ -418,11 +418,8 @@ __device__ __forceinline__ void row_scales(int fmt, float amax, float &s_x, floa
 
 // ---------------------------------------------------------------- kernel
 // Kernel modes. kRow: one second-level scale per row (written to row_scale). kSwiglu: as kRow,
-// the input formed as SiLU(g)*u from [g | u]. kAmax: only the row amax of xh, max-reduced into
-// row_scale[0] (float bits of a non-negative value order like unsigned integers). kTensor: the
-// second-level scale from the tensor amax left in row_scale[0] by kAmax; row_scale itself is
-// written afterwards by fill_row_scale (blocks still read row_scale[0] while others finish).
-constexpr int kRow = 0, kSwiglu = 1, kAmax = 2, kTensor = 3;
+// the input formed as SiLU(g)*u from [g | u].
+constexpr int kRow = 0, kSwiglu = 1;
 
 template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE, int DP>
 __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
@@ -495,11 +492,6 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
     }
   }
   am = team_max(am, W, team, wt, sm_f);
-  if (MODE == kAmax) {
-    if (live_row && wt == 0 && lane == 0) atomicMax(reinterpret_cast<unsigned int *>(p.row_scale), __float_as_uint(am));
-    return;
-  }
-  if (MODE == kTensor) am = p.row_scale[0];  // the tensor amax (kAmax pass)
   float s_x, g_x;
   row_scales(FMT, am, s_x, g_x);
 
@@ -530,20 +522,198 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
       store16<FMT, UNIT, DENSE>(chunk, o, 0u, 0u, 0u, 0u, 0u, 0u);
     }
   }
-  if (MODE != kTensor && live_row && wt == 0 && lane == 0) p.row_scale[row] = s_x;
+  if (live_row && wt == 0 && lane == 0) p.row_scale[row] = s_x;
 }
 
-// Per-tensor scale: every row's entry gets the NVFP4 scale of the tensor amax held in
-// row_scale[0] (one block; entry 0 is read before any is written).
-__global__ void __launch_bounds__(1024) fill_row_scale(float *row_scale, int T) {
-  __shared__ float s_x;
+// ---------------------------------------------------------------- one scale per tensor
+// NVFP4 with one second-level scale for the whole tensor needs the tensor amax before any code
+// is formed. One cooperative launch (every block resident at once): a block's teams take the
+// row groups blockIdx.x, blockIdx.x + G, ... Phase 1 loads each of its rows, forms rstd and the
+// normalized row amax; rstd waits in row_scale[row] for phase 2, except the last row's, which
+// stays in registers with the row itself. Each block writes its maximum to the workspace, a
+// grid barrier follows (an arrival counter the host cleared, a bounded wait), and every block
+// takes the maximum of all block maxima. Phase 2 quantizes the last row from registers and
+// re-reads the others, the most recently read first (L2 may still hold them); when every row
+// fits on chip (one row group per team) x is read once. Finally row_scale gets the tensor's
+// scale. Workspace words: [0] arrival counter, [1] barrier generation, [4 + b] block b's
+// maximum (float). The last block to arrive zeroes the counter and advances the generation,
+// so a call leaves the workspace ready for the next one (it starts from zeros).
+__device__ uint32_t g_prep_status = 0;  // bit 0: the grid barrier's wait gave up
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *a) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t *a) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+template <int UNIT, bool NORM, int DP>
+__global__ void __launch_bounds__(256, 2) prep_tensor_kernel(PrepParams p, uint32_t *ws, int groups,
+                                                          unsigned long long limit_ns) {
+  extern __shared__ float4 gamma_smem4[];
+  __shared__ double sm_d[64];
+  __shared__ float sm_f[64];
+  __shared__ float tensor_amax;
+  __shared__ int barrier_ok;
+  float *gs = reinterpret_cast<float *>(gamma_smem4);
+  const int W = p.TS;
+  const int teams = (blockDim.x >> 5) / W;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int team = warp / W, wt = warp - team * W;
+  const int ndp_row = p.K >> 4;
+  const int stride = 32 * W;
+  const int G = gridDim.x;
+  const int J = (groups - (int)blockIdx.x + G - 1) / G;  // >= 1: G <= groups
+  const float4 *g_lane = gamma_smem4 + wt * 128 + lane;
+
+  if (NORM) {
+    for (int k = 2 * threadIdx.x; k < p.K; k += 2 * blockDim.x) {
+      const uint32_t g2 = *reinterpret_cast<const uint32_t *>(p.gamma + k);
+      gs[gamma_smem_index(k)] = bf16lo(g2);
+      gs[gamma_smem_index(k + 1)] = bf16hi(g2);
+    }
+    __syncthreads();
+  }
+  uint32_t xr[DP][8];
+  auto load_row = [&](int row) {
+#pragma unroll
+    for (int i = 0; i < DP; ++i) {
+      const int dp = i * stride + wt * 32 + lane;
+      if (row < p.T && dp < ndp_row) ld256(p.x + (size_t)row * p.x_stride + (size_t)dp * 16, xr[i]);
+    }
+  };
+
+  // ---- phase 1: rstd and the normalized amax of every row of this block
+  float rstd = 1.f, am = 0.f;
+  for (int j = 0; j < J; ++j) {
+    const int row = ((int)blockIdx.x + j * G) * teams + team;
+    const bool live_row = row < p.T;
+    load_row(row);
+    if (NORM) {
+      double ss = 0.0;
+#pragma unroll
+      for (int i = 0; i < DP; ++i) {
+        const int dp = i * stride + wt * 32 + lane;
+        if (live_row && dp < ndp_row) {
+#pragma unroll
+          for (int w = 0; w < 8; ++w) ss = add_squares(xr[i][w], ss);
+        }
+      }
+      ss = team_sum(ss, W, team, wt, sm_d);
+      const float ms = __double2float_rn(__ddiv_rn(ss, (double)p.K));
+      rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, p.eps)));
+      if (j < J - 1 && live_row && wt == 0 && lane == 0) p.row_scale[row] = rstd;
+    }
+#pragma unroll
+    for (int i = 0; i < DP; ++i) {
+      const int dp = i * stride + wt * 32 + lane;
+      if (live_row && dp < ndp_row) {
+        float v[16];
+        unpack16(xr[i], v);
+        if (NORM) normalize16<true>(v, g_lane + i * 128 * W, rstd);
+        am = amax16(v, am);
+      }
+    }
+  }
+
+  // ---- block maximum, grid barrier, tensor maximum
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(kFull, am, o));
+  if (lane == 0) sm_f[warp] = am;
+  __syncthreads();
+  float *bmax = reinterpret_cast<float *>(ws + 4);
   if (threadIdx.x == 0) {
-    float s, g;
-    row_scales(kFmtNV, row_scale[0], s, g);
-    s_x = s;
+    float m = sm_f[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, sm_f[w]);
+    // generation read before arriving: it advances only after every block has arrived
+    const uint32_t gen = ld_relaxed_gpu(ws + 1);
+    bmax[blockIdx.x] = m;
+    __threadfence();
+    bool ok = true;
+    if (atomicAdd(ws, 1u) == (uint32_t)G - 1u) {
+      // the last block: reset the counter for the next call, then release the others
+      atomicExch(ws, 0u);
+      __threadfence();
+      atomicAdd(ws + 1, 1u);
+    } else if (ld_acquire_gpu(ws + 1) == gen) {
+      ok = false;
+      const uint64_t t0 = global_ns();
+      for (uint32_t i = 1;; ++i) {
+        if (ld_acquire_gpu(ws + 1) != gen) { ok = true; break; }
+        if ((i & 31u) == 0 && global_ns() - t0 > limit_ns) break;
+      }
+    }
+    if (!ok) atomicOr(&g_prep_status, 1u);
+    barrier_ok = ok ? 1 : 0;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < T; i += blockDim.x) row_scale[i] = s_x;
+  if (!barrier_ok) return;  // outputs undefined; the status word reports it
+  // the maximum of the G block maxima, read by the whole block at once
+  float t = 0.f;
+  for (int b = threadIdx.x; b < G; b += blockDim.x) t = fmaxf(t, __ldcg(bmax + b));
+  for (int o = 16; o > 0; o >>= 1) t = fmaxf(t, __shfl_xor_sync(kFull, t, o));
+  __syncthreads();  // sm_f's block maxima have been read
+  if (lane == 0) sm_f[warp] = t;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = sm_f[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, sm_f[w]);
+    tensor_amax = m;
+  }
+  __syncthreads();
+  float s_x, g_x;
+  row_scales(kFmtNV, tensor_amax, s_x, g_x);
+
+  // ---- phase 2: quantize, the row still in registers first
+  constexpr int kChunk = act_tile(kFmtNV, UNIT, true).bytes;
+  for (int j = J - 1; j >= 0; --j) {
+    const int row = ((int)blockIdx.x + j * G) * teams + team;
+    const bool live_row = row < p.T;
+    if (j < J - 1) {
+      load_row(row);
+      if (NORM) rstd = live_row ? __ldcg(p.row_scale + row) : 1.f;
+    }
+    const Spot o = lane_spot<kFmtNV, UNIT, false>(row, lane);
+    uint8_t *chunk0 = p.tiles + ((size_t)(row >> 7) * p.KS + 2 * wt + (lane >> 4)) * kChunk;
+    const size_t chunk_step = (size_t)2 * W * kChunk;
+    const bool pad_row = !live_row && row < p.T_pad;
+#pragma unroll
+    for (int i = 0; i < DP; ++i) {
+      const int base = i * stride + wt * 32;  // warp-uniform
+      if (base >= ndp_row) break;
+      const int dp = base + lane;
+      const bool live = live_row && dp < ndp_row;
+      uint8_t *chunk = chunk0 + i * chunk_step;
+      if (live_row) {
+        float v[16];
+        if (live) {
+          unpack16(xr[i], v);
+          if (NORM) normalize16<false>(v, g_lane + i * 128 * W, rstd);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) v[q] = 0.f;
+        }
+        process16<kFmtNV, UNIT, false>(chunk, o, v, live, s_x, g_x);
+      } else if (pad_row && dp < ndp_row) {
+        store16<kFmtNV, UNIT, false>(chunk, o, 0u, 0u, 0u, 0u, 0u, 0u);
+      }
+    }
+  }
+  __syncthreads();  // every warp of a team has read its rows' rstd before the entries change
+  for (int j = 0; j < J; ++j) {
+    const int row = ((int)blockIdx.x + j * G) * teams + team;
+    if (row < p.T && wt == 0 && lane == 0) p.row_scale[row] = s_x;
+  }
 }
 
 template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE, int DP>
@@ -608,23 +778,68 @@ cudaError_t launch_prep(PrepParams p, int fmt, int unit, bool norm, bool dense, 
   return unit == 2 ? launch_n<kFmtMX, 2, false>(p, norm, st) : launch_n<kFmtMX, 1, false>(p, norm, st);
 }
 
-// NVFP4 with one second-level scale for the whole tensor: tensor amax (clear + one pass),
-// the preparation with that scale, then the per-row copies of the scale.
-cudaError_t launch_prep_tensor_scale(PrepParams p, int unit, bool norm, cudaStream_t st) {
+// Row groups of the per-tensor launch: teams of TS warps, 8 warps per block.
+int prep_tensor_groups(int tokens, int k) {
+  const int ts = prep_team_warps(k);
+  const int teams = ts >= 8 ? 1 : 8 / ts;
+  return (round_up(tokens, 256) + teams - 1) / teams;
+}
+
+namespace {
+template <int UNIT, bool NORM, int DP>
+cudaError_t launch_tensor_t(PrepParams p, uint32_t *ws, unsigned long long limit_ns, cudaStream_t st) {
+  auto kern = prep_tensor_kernel<UNIT, NORM, DP>;
+  static std::once_flag once[64];
+  static cudaError_t err[64];
+  static int sms[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [dev, kern] {
+    err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 * (int)sizeof(float));
+    if (err[dev] == cudaSuccess) err[dev] = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+  });
+  if (err[dev] != cudaSuccess) return err[dev];
+  const int W = p.TS;
+  const int teams = W >= 8 ? 1 : 8 / W;
+  const int block = teams * W * 32;
+  const size_t smem = NORM ? (size_t)((p.K + 511) / 512 * 512) * sizeof(float) : 0;
+  int per_sm = 0;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, block, smem)) != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+  int groups = (p.T_pad + teams - 1) / teams;
+  const int grid = groups < per_sm * sms[dev] ? groups : per_sm * sms[dev];
+  void *args[] = {&p, &ws, &groups, &limit_ns};
+  e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), dim3(grid), dim3(block), args, smem, st);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int UNIT, bool NORM>
+cudaError_t launch_tensor_dp(const PrepParams &p, uint32_t *ws, unsigned long long limit_ns, cudaStream_t st) {
+  if (p.TS == 1 && p.K / 16 <= 32 * 4) return launch_tensor_t<UNIT, NORM, 4>(p, ws, limit_ns, st);
+  return launch_tensor_t<UNIT, NORM, kMaxDP>(p, ws, limit_ns, st);
+}
+}  // namespace
+
+// NVFP4 with one second-level scale for the whole tensor: one cooperative launch.
+cudaError_t launch_prep_tensor_scale(PrepParams p, int unit, bool norm, void *workspace, unsigned long long limit_ns,
+                                     cudaStream_t st) {
   p.KS = p.K / 256;
   p.TS = prep_team_warps(p.K);
   if (p.TS > 8) return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(p.row_scale, 0, sizeof(float), st);
-  if (e != cudaSuccess) return e;
-  e = norm ? launch_t<kFmtNV, 2, true, false, kAmax>(p, st) : launch_t<kFmtNV, 2, false, false, kAmax>(p, st);
-  if (e != cudaSuccess) return e;
+  uint32_t *ws = static_cast<uint32_t *>(workspace);
   if (unit == 2)
-    e = norm ? launch_t<kFmtNV, 2, true, false, kTensor>(p, st) : launch_t<kFmtNV, 2, false, false, kTensor>(p, st);
-  else
-    e = norm ? launch_t<kFmtNV, 1, true, false, kTensor>(p, st) : launch_t<kFmtNV, 1, false, false, kTensor>(p, st);
+    return norm ? launch_tensor_dp<2, true>(p, ws, limit_ns, st) : launch_tensor_dp<2, false>(p, ws, limit_ns, st);
+  return norm ? launch_tensor_dp<1, true>(p, ws, limit_ns, st) : launch_tensor_dp<1, false>(p, ws, limit_ns, st);
+}
+
+cudaError_t read_and_clear_prep_status(uint32_t *status) {
+  uint32_t zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(status, g_prep_status, sizeof *status);
   if (e != cudaSuccess) return e;
-  fill_row_scale<<<1, 1024, 0, st>>>(p.row_scale, p.T);
-  return cudaGetLastError();
+  return cudaMemcpyToSymbol(g_prep_status, &zero, sizeof zero);
 }
 
 }  // namespace sharq

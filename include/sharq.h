@@ -154,13 +154,27 @@ int sharq_prepare(const void *x_bf16_dev, int tokens, int k, const void *gamma_b
 /* sharq_prepare with ONE NVFP4 second-level scale for the whole activation tensor instead
  * of one per row: s_x = fp32(amax|xh|/2688) over every row (the stricter reading of NVFP4's
  * "fp32 tensor scale"), shared by backbone and residual; row_scale receives that value in
- * every entry, so sharq_linear consumes the result unchanged. Three launches (a tensor-amax
- * pass over x, the preparation, a fill of row_scale) plus a 4-byte clear of row_scale[0],
- * which holds the tensor amax in between. MXFP4 has no second-level scale: same as
- * sharq_prepare. Arguments, layouts and errors as sharq_prepare. */
+ * every entry, so sharq_linear consumes the result unchanged. MXFP4 has no second-level
+ * scale: same as sharq_prepare (the workspace is not touched).
+ * One cooperative launch (every block resident): a first phase forms each row's rstd and
+ * normalized amax (rstd is parked in row_scale), a grid-wide barrier exchanges the block maxima
+ * through the workspace, a second phase quantizes. When every row fits on chip (about 2400
+ * rows at k = 4096 on B200) x is read once; beyond that the rows not held in registers are
+ * read again, the most recent first.
+ *   workspace_dev  caller-owned device buffer of sharq_tensor_scale_workspace_size(tokens, k)
+ *                  bytes, 16-byte aligned, ZEROED ONCE before its first use (e.g. by
+ *                  cudaMemset when it is allocated). Each call leaves its barrier words ready
+ *                  for the next, so it can be reused without clearing, across sizes too
+ *                  (a buffer sized for the largest call serves all). Calls whose launches may
+ *                  overlap on the GPU need distinct workspaces.
+ * If the barrier's bounded wait gives up (only if blocks were not all resident), the call's
+ * outputs are undefined, sharq_device_status reports SHARQ_ERR_TIMEOUT, and the workspace
+ * must be zeroed again before it is reused. Other arguments, layouts and errors as
+ * sharq_prepare. */
+size_t sharq_tensor_scale_workspace_size(int tokens, int k);
 int sharq_prepare_tensor_scale(const void *x_bf16_dev, int tokens, int k, const void *gamma_bf16_dev,
                                float eps, int nm_n, int nm_m, int unit, int fmt, sharq_prep *out,
-                               void *stream);
+                               void *workspace_dev, void *stream);
 
 /* The preparation operator fed by a gate/up projection's output (one launch): the down
  * projection's input x = SiLU(g) * u is formed in registers from [g | u] and prepared as
@@ -239,9 +253,9 @@ int sharq_mma_peak(int mode, int fmt, int iters, int clusters, void *stream);
  * bounded waits set when they give up: SHARQ_OK or SHARQ_ERR_TIMEOUT (or SHARQ_ERR_CUDA). */
 int sharq_device_status(void *stream);
 
-/* Test hook: time limit, in nanoseconds, of the GEMM's bounded waits (0 restores the
- * default of 4 s). Process-wide (one atomic value shared by every host thread), read by
- * each GEMM call when it launches. Lowering it lets a test make a wait give up without faulting the device:
+/* Test hook: time limit, in nanoseconds, of the GEMM's bounded waits and of the per-tensor
+ * preparation's grid barrier (0 restores the default of 4 s). Process-wide (one atomic value
+ * shared by every host thread), read by each call when it launches. Lowering it lets a test make a wait give up without faulting the device:
  * the kernel records SHARQ_ERR_TIMEOUT, drains its own copies and MMAs, frees its tensor
  * memory and returns; its output is then undefined. Applies to calls issued afterwards. */
 void sharq_set_wait_limit(long long nanoseconds);

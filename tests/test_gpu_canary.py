@@ -84,8 +84,10 @@ def test_no_writes_outside_buffers(fmt, T, K, N):
     S.sharq_prepare_swiglu(gu, 2, 4, 2, fmt, out=p)
     guards += gp
     p, gp = guarded_prep(S, T, K, 2, fmt)
-    S.sharq_prepare_tensor_scale(x, g, 1e-6, 2, 4, 2, fmt, out=p)
-    guards += gp
+    gw = Guarded(S.sharq_tensor_scale_workspace_size(T, K))
+    gw.view.zero_()
+    S.sharq_prepare_tensor_scale(x, g, 1e-6, 2, 4, 2, fmt, out=p, workspace=gw.view)
+    guards += list(gp) + [gw]
     s = S.sharq_dense_buffer_sizes(T, K, fmt)
     gt, gr = Guarded(s[0]), Guarded(s[1])
     q = S.DenseQ(gt.view, gr.as_type(torch.float32, (T,)), T, K, S._fmt(fmt))

@@ -70,3 +70,32 @@ def test_zero_tensor():
     got = hw.read_prep(p, 16)
     assert np.all(got["row_scale"] == 1.0)
     assert not got["sp_codes"].any() and not got["res_codes"].any()
+
+
+@pytest.mark.parametrize("T,K,norm", [(5000, 256, False), (1500, 8192, False), (3000, 4096, True)])
+def test_tensor_scale_several_row_groups_per_block(T, K, norm):
+    """More row groups than resident blocks: phase 2 re-reads rows (and their parked rstd)."""
+    S = require_gpu()
+    rng = np.random.default_rng(T + K)
+    x_bits = wl.outlier_activations(rng, T, K, max(2, K // 100), 20.0, 100.0, 0.5)
+    g_bits = wl.rms_gamma(rng, K) if norm else None
+    ws = torch.zeros(S.sharq_tensor_scale_workspace_size(T, K), dtype=torch.uint8, device="cuda")
+    x = to_dev_bf16(x_bits)
+    g = to_dev_bf16(g_bits) if norm else None
+    p = S.sharq_prepare_tensor_scale(x, g, 1e-6, workspace=ws)
+    p2 = S.sharq_prepare_tensor_scale(x, g, 1e-6, workspace=ws)  # the same workspace again
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0  # the counter is left at zero
+    assert int(ws[4:8].view(torch.int32).item()) == 2  # two barrier generations
+    assert S.sharq_device_status() == S.SHARQ_OK
+    assert torch.equal(p.tiles, p2.tiles) and torch.equal(p.row_scale, p2.row_scale)
+    got = hw.read_prep(p, 16)
+    ref = O.prepare(f32(x_bits), f32(g_bits) if norm else None, 1e-6, 2, 4, 2, O.NVFP4, per_tensor=True)
+    assert np.all(got["row_scale"] == got["row_scale"][0])
+    if not norm:
+        for key in KEYS:
+            assert np.array_equal(got[key], ref[key]), key
+    else:
+        assert abs(int(got["row_scale"][0].view(np.int32)) - int(ref["row_scale"][0].view(np.int32))) <= 1
+        for key in ("sp_codes", "res_codes", "idx"):
+            assert np.mean(got[key] != ref[key]) <= 1e-4, key
