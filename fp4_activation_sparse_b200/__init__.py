@@ -66,6 +66,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sharq_wpack_buffer_sizes": (S, [I, I, I, ctypes.POINTER(S)]),
         "sharq_pack_weight": (I, [P, I, I, I, ctypes.POINTER(_WPack), P]),
         "sharq_prepare": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P]),
+        "sharq_prepare_tensor_scale_noalloc": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P]),
         "sharq_prepare_swiglu": (I, [P, I, I, I, I, I, I, ctypes.POINTER(_Prep), P]),
         "sharq_tensor_scale_workspace_size": (S, [I, I]),
         "sharq_prepare_tensor_scale": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P, P]),
@@ -250,6 +251,23 @@ def sharq_prepare_tensor_scale(x: torch.Tensor, gamma: torch.Tensor | None = Non
     st = out.struct()
     _check(lib.sharq_prepare_tensor_scale(_ptr(x), tokens, k, _ptr(gamma), ctypes.c_float(eps), nm_n, nm_m, unit,
                                           _fmt(fmt), ctypes.byref(st), _ptr(workspace), _stream(stream)))
+    return out
+
+
+def sharq_prepare_tensor_scale_noalloc(x: torch.Tensor, gamma: torch.Tensor | None = None, eps: float = 1e-6,
+                                       nm_n: int = 2, nm_m: int = 4, unit: int = UNIT_PAIR, fmt="nvfp4",
+                                       out: Prep | None = None, stream=None) -> Prep:
+    """sharq_prepare_tensor_scale without a workspace: for callers that may not allocate device
+    memory, the library's own static scratch carries the grid barrier (calls that overlap on the
+    GPU race on it). Only the output holder is allocated here, and only if `out` is omitted."""
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous()
+    tokens, k = x.shape
+    if gamma is not None:
+        assert gamma.dtype == torch.bfloat16 and gamma.is_cuda and gamma.numel() == k
+    out = out or alloc_prep(tokens, k, nm_n, nm_m, unit, fmt, x.device)
+    st = out.struct()
+    _check(lib.sharq_prepare_tensor_scale_noalloc(_ptr(x), tokens, k, _ptr(gamma), ctypes.c_float(eps), nm_n, nm_m,
+                                                  unit, _fmt(fmt), ctypes.byref(st), _stream(stream)))
     return out
 
 

@@ -189,6 +189,52 @@ int sharq_prepare_tensor_scale(const void *x, int tokens, int k, const void *gam
   return s;
 }
 
+int sharq_prepare_tensor_scale_noalloc(const void *x, int tokens, int k, const void *gamma, float eps, int nm_n,
+                                       int nm_m, int unit, int fmt, sharq_prep *out, void *stream) {
+  if (!out) return fail(SHARQ_ERR_INVALID_ARG, "output struct is null");
+  if (int s = check_pattern(nm_n, nm_m, unit)) return s;
+  if (fmt != SHARQ_NVFP4)  // MXFP4 has no second-level scale: the per-row operator, no scratch
+    return sharq_prepare(x, tokens, k, gamma, eps, nm_n, nm_m, unit, fmt, out, stream);
+  if (!x) return fail(SHARQ_ERR_INVALID_ARG, "x is null");
+  if (int s = check_shape(tokens, k, "tokens")) return s;
+  if (k > 32768) return fail(SHARQ_ERR_INVALID_ARG, "k must be <= 32768 for the preparation kernel (got %d)", k);
+  if (((uintptr_t)x & 31u) || ((uintptr_t)gamma & 31u))
+    return fail(SHARQ_ERR_INVALID_ARG, "x and gamma must be 32-byte aligned (256-bit loads)");
+  if (!out->tiles || !out->row_scale) return fail(SHARQ_ERR_INVALID_ARG, "null output buffer");
+  if (!aligned16(out->tiles) || !aligned16(out->row_scale))
+    return fail(SHARQ_ERR_INVALID_ARG, "output buffers must be 16-byte aligned");
+  if (gamma && !(eps >= 0.f)) return fail(SHARQ_ERR_INVALID_ARG, "eps must be >= 0");
+  sharq::PrepParams p;
+  memset(&p, 0, sizeof p);
+  p.x = static_cast<const uint16_t *>(x);
+  p.x_stride = k;
+  p.gamma = static_cast<const uint16_t *>(gamma);
+  p.eps = eps;
+  p.T = tokens;
+  p.K = k;
+  p.T_pad = sharq::round_up(tokens, 256);
+  p.tiles = static_cast<uint8_t *>(out->tiles);
+  p.row_scale = out->row_scale;
+  const long long lim = g_wait_limit.load(std::memory_order_relaxed);
+  size_t needed = 0, capacity = 0;
+  cudaError_t e = sharq::launch_prep_tensor_scale_static(p, unit, gamma != nullptr,
+                                                         lim > 0 ? (unsigned long long)lim : 4000000000ull,
+                                                         static_cast<cudaStream_t>(stream), &needed, &capacity);
+  if (e == cudaErrorInvalidValue && needed > capacity)
+    return fail(SHARQ_ERR_UNSUPPORTED, "sharq_prepare_tensor_scale_noalloc: this launch needs %zu bytes of scratch, "
+                "the library's static scratch holds %zu (use sharq_prepare_tensor_scale with a workspace)",
+                needed, capacity);
+  if (e != cudaSuccess) return cuda_fail(e, "sharq_prepare_tensor_scale_noalloc");
+  out->tokens = tokens;
+  out->k = k;
+  out->nm_n = nm_n;
+  out->nm_m = nm_m;
+  out->unit = unit;
+  out->fmt = fmt;
+  g_err[0] = 0;
+  return SHARQ_OK;
+}
+
 int sharq_prepare_swiglu(const void *gate_up, int tokens, int k, int nm_n, int nm_m, int unit, int fmt,
                          sharq_prep *out, void *stream) {
   if (!out) return fail(SHARQ_ERR_INVALID_ARG, "output struct is null");

@@ -88,6 +88,8 @@ cudaError_t launch_prep(PrepParams p, int fmt, int unit, bool norm, bool dense, 
 cudaError_t launch_prep_tensor_scale(PrepParams p, int unit, bool norm, void *workspace, unsigned long long limit_ns,
                                      cudaStream_t st);
 int prep_tensor_groups(int tokens, int k);
+cudaError_t launch_prep_tensor_scale_static(PrepParams p, int unit, bool norm, unsigned long long limit_ns,
+                                            cudaStream_t st, size_t *needed, size_t *capacity);
 cudaError_t read_and_clear_prep_status(uint32_t *status);
 cudaError_t launch_pack(PackParams p, int fmt, cudaStream_t st);
 cudaError_t launch_gemm(GemmParams p, cudaStream_t st, const char **why);

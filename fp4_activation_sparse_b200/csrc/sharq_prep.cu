@@ -835,6 +835,49 @@ cudaError_t launch_prep_tensor_scale(PrepParams p, int unit, bool norm, void *wo
   return norm ? launch_tensor_dp<1, true>(p, ws, limit_ns, st) : launch_tensor_dp<1, false>(p, ws, limit_ns, st);
 }
 
+// ---------------------------------------------------------------- per-tensor scale, no caller memory
+// The per-tensor preparation for callers that cannot hand the library a workspace: code that
+// runs where it may not allocate device memory at all (inside a memory budget owned by a host
+// framework or an inference server that pre-assigns every byte, or a plugin ABI that passes
+// only its tensors), or where cudaMalloc's implicit device synchronization would stall a
+// latency-critical path. The grid barrier's words and block maxima live in this file-scope
+// array instead, loaded with the library and held by every GPU that loads it until exit.
+// One array per device, shared by every call on that device: calls whose launches may overlap
+// on the GPU (different streams, no ordering between them) race on it.
+namespace {
+constexpr size_t kStaticScratchBytes = 8192;  // barrier words + up to 2044 block maxima
+static __device__ __align__(256) uint32_t g_static_scratch[kStaticScratchBytes / 4];
+}  // namespace
+
+cudaError_t launch_prep_tensor_scale_static(PrepParams p, int unit, bool norm, unsigned long long limit_ns,
+                                            cudaStream_t st, size_t *needed, size_t *capacity) {
+  // Once per device, with that device current: the array's device address. In host code the
+  // array's name is only a host-side stand-in, never a pointer a kernel may be given.
+  static std::once_flag once[64];
+  static cudaError_t err[64];
+  static void *addr[64];
+  static int sms[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [dev] {
+    err[dev] = cudaGetSymbolAddress(&addr[dev], g_static_scratch);
+    if (err[dev] == cudaSuccess) err[dev] = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+  });
+  if (err[dev] != cudaSuccess) return err[dev];
+  // the launch uses at most one block slot per row group and at most 8 resident blocks of 256
+  // threads per SM
+  const int groups = prep_tensor_groups(p.T, p.K);
+  const int max_grid = 8 * sms[dev];
+  *needed = 16 + 4 * (size_t)(groups < max_grid ? groups : max_grid);
+  *capacity = kStaticScratchBytes;
+  if (*needed > kStaticScratchBytes) return cudaErrorInvalidValue;
+  // the array keeps the previous call's contents: the counter and generation start at zero
+  if ((e = cudaMemsetAsync(addr[dev], 0, 2 * sizeof(uint32_t), st)) != cudaSuccess) return e;
+  return launch_prep_tensor_scale(p, unit, norm, addr[dev], limit_ns, st);
+}
+
 cudaError_t read_and_clear_prep_status(uint32_t *status) {
   uint32_t zero = 0;
   cudaError_t e = cudaMemcpyFromSymbol(status, g_prep_status, sizeof *status);

@@ -176,6 +176,28 @@ int sharq_prepare_tensor_scale(const void *x_bf16_dev, int tokens, int k, const 
                                float eps, int nm_n, int nm_m, int unit, int fmt, sharq_prep *out,
                                void *workspace_dev, void *stream);
 
+/* sharq_prepare_tensor_scale for callers that cannot allocate device memory. The paper has no
+ * counterpart: this is an integration variant. Some callers may not call cudaMalloc at all --
+ * a host framework or inference server that owns every byte of the GPU's memory and hands a
+ * kernel library only its tensors, or a latency-critical path where cudaMalloc's implicit
+ * device synchronization is not acceptable -- so they have no way to supply the workspace.
+ * This entry point allocates nothing: the grid barrier's words and the block maxima live in a
+ * static device array of 8192 bytes inside the library (held on every GPU that loads the
+ * library until the process exits), enough for launches of up to 2044 blocks; a launch that
+ * would need more (a GPU with more than 255 SMs) is rejected with SHARQ_ERR_UNSUPPORTED and a
+ * message naming both sizes, and nothing is launched. The caller still passes the input and
+ * the output struct; results are identical to sharq_prepare_tensor_scale's.
+ *   - Every call on a device shares that array, and it keeps the last call's contents: each
+ *     call clears its barrier words on `stream` first (an 8-byte memset, no allocation). Calls
+ *     whose launches may overlap on the GPU race on the array: order them on one stream.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current) and caches it; make that first call before any stream capture.
+ *   - MXFP4 has no second-level scale: as sharq_prepare, the array is not touched.
+ * Arguments, layouts and errors otherwise as sharq_prepare_tensor_scale. */
+int sharq_prepare_tensor_scale_noalloc(const void *x_bf16_dev, int tokens, int k, const void *gamma_bf16_dev,
+                                       float eps, int nm_n, int nm_m, int unit, int fmt, sharq_prep *out,
+                                       void *stream);
+
 /* The preparation operator fed by a gate/up projection's output (one launch): the down
  * projection's input x = SiLU(g) * u is formed in registers from [g | u] and prepared as
  * by sharq_prepare without normalization, so x never goes through memory (the abstract's
