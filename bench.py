@@ -528,6 +528,30 @@ def run_sharq(args, rank, world, local):
                 "prep_gbs": pb / (tp / 1e3) / 1e9, "prep_frac": pb / (tp / 1e3) / 1e9 / hbm_peak,
                 "l2": f"{n} rotating set(s)"}
 
+    def measure_prep_only(name, T_, K_, fmt, nm, seed):
+        """A mask pattern no sparse FP4 MMA executes (elements 2:4, elements 4:8): the
+        preparation alone, same rotation rule."""
+        n_, m_, unit_ = nm
+        blk = 16 if fmt == "nvfp4" else 32
+        meta = (3.0 / 16 if m_ == 8 else 1.0 / 8 if unit_ == 1 else 1.0 / 16)  # metadata bytes per element
+        pb_elem = 2 + 0.25 + meta + 0.5 / blk + 0.5 + 1 / blk
+        n = int(min(32, max(1, np.ceil(3 * L2_BYTES / (T_ * K_ * pb_elem)))))
+        x0 = wl.outlier_activations_device(seed, T_, K_, max(1, K_ // 100), 20.0, 100.0, 0.5)
+        xs_ = [x0] + [x0.clone() for _ in range(n - 1)]
+        ps = [S.alloc_prep(T_, K_, n_, m_, unit_, fmt) for _ in range(n)]
+
+        def prep_all(st):
+            for i in range(n):
+                S.sharq_prepare(xs_[i], None, 1e-6, n_, m_, unit_, fmt, out=ps[i], stream=st)
+
+        prep_all(stream)
+        torch.cuda.synchronize()
+        tp = graph_time(capture(prep_all), n)
+        pb = T_ * K_ * pb_elem + T_ * 4
+        return {"workload": name, "T": T_, "K": K_, "fmt": fmt, "pattern": f"{n_}:{m_} over {'pairs' if unit_ == 2 else 'elements'}",
+                "executed_by_sharq_linear": False, "t_prep_us": tp * 1e3, "prep_gbs": pb / (tp / 1e3) / 1e9,
+                "prep_frac": pb / (tp / 1e3) / 1e9 / hbm_peak, "l2": f"{n} rotating set(s)"}
+
     sweep = []
     if not args.no_sweep:
         cases = [("llama31_8b_qkv_prefill", 16384, 4096, 6144, True, "nvfp4", False),
@@ -541,6 +565,10 @@ def run_sharq(args, rank, world, local):
             cases.append(("video_dit", 32760, 5120, 5120, False, fmt_, False))
         for ci, c in enumerate(cases):
             sweep.append(measure_linear(*c[:6], seed=9000 + 10 * ci, swiglu_input=c[6]))
+        for fmt_ in ("nvfp4", "mxfp4"):
+            for nm in ((4, 8, 1), (2, 4, 1)):
+                sweep.append(measure_prep_only("square_8192", 8192, 8192, fmt_, nm, 9700))
+                sweep.append(measure_prep_only("video_dit", 32760, 5120, fmt_, nm, 9710))
         assert S.sharq_device_status() == S.SHARQ_OK
 
     # ---- end to end through the public API with host buffers: every step copies its input

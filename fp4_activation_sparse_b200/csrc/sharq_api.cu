@@ -43,6 +43,17 @@ int check_pattern(int nm_n, int nm_m, int unit) {
   return 0;
 }
 
+// sharq_prepare and the size query also take four of eight elements (4:8, unit 1); returns 0
+// or a status and sets *code to the layout's pattern code (2 pairs, 1 elements 2:4, kPat48).
+int check_prepare_pattern(int nm_n, int nm_m, int unit, int *code) {
+  if (nm_n == 4 && nm_m == 8 && unit == 1) {
+    *code = sharq::kPat48;
+    return 0;
+  }
+  *code = unit;
+  return check_pattern(nm_n, nm_m, unit);
+}
+
 int check_shape(int rows, int k, const char *rows_name) {
   if (rows < 1) return fail(SHARQ_ERR_INVALID_ARG, "%s must be >= 1 (got %d)", rows_name, rows);
   if (k < 256 || k % 256 != 0) return fail(SHARQ_ERR_INVALID_ARG, "k must be a positive multiple of 256 (got %d)", k);
@@ -63,8 +74,9 @@ void sharq_set_wait_limit(long long nanoseconds) { g_wait_limit.store(nanosecond
 size_t sharq_prep_buffer_sizes(int tokens, int k, int nm_n, int nm_m, int unit, int fmt, size_t sizes[2]) {
   if (!sizes) { fail(SHARQ_ERR_INVALID_ARG, "sizes is null"); return 0; }
   if (!valid_fmt(fmt)) { fail(SHARQ_ERR_INVALID_ARG, "unknown fmt %d", fmt); return 0; }
-  if (check_shape(tokens, k, "tokens") || check_pattern(nm_n, nm_m, unit)) return 0;
-  const sharq::ActTile A = sharq::act_tile(fmt, unit, true);
+  int code = 0;
+  if (check_shape(tokens, k, "tokens") || check_prepare_pattern(nm_n, nm_m, unit, &code)) return 0;
+  const sharq::ActTile A = sharq::act_tile(fmt, code, true);
   sizes[0] = (size_t)(sharq::round_up(tokens, 256) / 128) * (k / 256) * A.bytes;  // tiles
   sizes[1] = (size_t)tokens * 4;                                                    // row scales
   return sizes[0] + sizes[1];
@@ -150,8 +162,9 @@ static int prepare_common(const void *x, int tokens, int k, const void *gamma, f
 int sharq_prepare(const void *x, int tokens, int k, const void *gamma, float eps, int nm_n, int nm_m, int unit,
                   int fmt, sharq_prep *out, void *stream) {
   if (!out) return fail(SHARQ_ERR_INVALID_ARG, "output struct is null");
-  if (int s = check_pattern(nm_n, nm_m, unit)) return s;
-  int s = prepare_common(x, tokens, k, gamma, eps, fmt, false, unit, static_cast<uint8_t *>(out->tiles),
+  int code = 0;
+  if (int s = check_prepare_pattern(nm_n, nm_m, unit, &code)) return s;
+  int s = prepare_common(x, tokens, k, gamma, eps, fmt, false, code, static_cast<uint8_t *>(out->tiles),
                          out->row_scale, static_cast<cudaStream_t>(stream));
   if (s == SHARQ_OK) {
     out->tokens = tokens;

@@ -32,10 +32,16 @@ __host__ __device__ constexpr int tile_round(int a) { return (a + 1023) / 1024 *
 // scale atoms (512 B, 4 scales x 128 rows) per 256-K step for 128 rows; fmt 0 = NVFP4, 1 = MXFP4
 __host__ __device__ constexpr int atoms_res(int fmt) { return fmt == 0 ? 4 : 2; }  // one scale per B
 __host__ __device__ constexpr int atoms_sp(int fmt) { return fmt == 0 ? 2 : 1; }   // one scale per 2B
+// Mask pattern codes (the `unit` argument of the layout and the preparation's templates):
+// 2 = two of four pairs, 1 = two of four elements, kPat48 = four of eight elements.
+constexpr int kPat48 = 3;
+// metadata bytes per chunk: 128 rows x 16 B (pairs: 4-bit entries per 8 elements), x 32 B
+// (elements 2:4: 4 bits per 4), x 48 B (elements 4:8: 12 bits per 8)
+__host__ __device__ constexpr int meta_bytes(int unit) { return unit == 2 ? 2048 : unit == 1 ? 4096 : 6144; }
 __host__ __device__ constexpr ActTile act_tile(int fmt, int unit, bool sparse) {
-  return sparse ? ActTile{0, 16384, 24576, 24576 + (unit == 2 ? 2048 : 4096),
-                          24576 + (unit == 2 ? 2048 : 4096) + 512 * atoms_sp(fmt),
-                          tile_round(24576 + (unit == 2 ? 2048 : 4096) + 512 * (atoms_sp(fmt) + atoms_res(fmt)))}
+  return sparse ? ActTile{0, 16384, 24576, 24576 + meta_bytes(unit),
+                          24576 + meta_bytes(unit) + 512 * atoms_sp(fmt),
+                          tile_round(24576 + meta_bytes(unit) + 512 * (atoms_sp(fmt) + atoms_res(fmt)))}
                 : ActTile{0, 0, 0, 0, 16384, tile_round(16384 + 512 * atoms_res(fmt))};
 }
 __host__ __device__ constexpr WTile w_tile(int fmt) {

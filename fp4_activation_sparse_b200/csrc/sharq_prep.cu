@@ -53,6 +53,25 @@ __device__ __forceinline__ uint32_t top2_of_4(float k0, float k1, float k2, floa
   return min(first, second) | (max(first, second) << 2);
 }
 
+// The four largest of eight keys, ties to the lower index, as a bit mask (bit i: key i kept).
+// Key i is kept when fewer than four keys beat it: key j beats key i when it is larger, or
+// equal with j < i. Each of the 28 pairs is compared once.
+__device__ __forceinline__ uint32_t top4_of_8(const float *a) {
+  int beaten[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = i + 1; j < 8; ++j) {
+      const int jb = a[j] > a[i] ? 1 : 0;  // the higher index wins only when strictly larger
+      beaten[i] += jb;
+      beaten[j] += 1 - jb;
+    }
+  uint32_t keep = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) keep |= (beaten[i] < 4 ? 1u : 0u) << i;
+  return keep;
+}
+
 // ---------------------------------------------------------------- I/O
 __device__ __forceinline__ void ld256(const void *p, uint32_t (&r)[8]) {
   asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
@@ -252,6 +271,7 @@ __device__ __forceinline__ void deq8(uint32_t w, float dec, float s_x, float *o)
 // the chunk changes from piece to piece.
 struct Spot {
   int res, sp, meta, sf_sp, sf_res;  // byte offsets inside a chunk (sf_*: -1 = no scale byte here)
+  int mb;                            // elements 4:8: first metadata byte of the lane in its row
 };
 template <int FMT, int UNIT, bool DENSE>
 __device__ __forceinline__ Spot lane_spot(int row, int lane) {
@@ -262,7 +282,11 @@ __device__ __forceinline__ Spot lane_spot(int row, int lane) {
   o.res = L.res + r * 128 + (((j >> 1) ^ (r & 7)) << 4) + (j & 1) * 8;
   // 64-byte rows, 16-byte unit j/4 swizzled with row bits 1..2
   o.sp = L.sp + r * 64 + (((j >> 2) ^ ((r >> 1) & 3)) << 4) + (j & 3) * 4;
-  o.meta = UNIT == 2 ? L.meta + r * 16 + j : L.meta + (j >> 3) * 2048 + r * 16 + (j & 7) * 2;
+  // pairs: byte j of the row's 16; elements 2:4: 2 bytes at 2j of 32 (halves of 16 B 2048 apart);
+  // elements 4:8: 3 bytes from 3j of 48 (thirds of 16 B 2048 apart; store16 places each byte)
+  o.meta = UNIT == 2 ? L.meta + r * 16 + j
+                     : UNIT == 1 ? L.meta + (j >> 3) * 2048 + r * 16 + (j & 7) * 2 : L.meta + r * 16;
+  o.mb = 3 * j;
   if (FMT == kFmtNV) {  // one backbone scale per 2 pieces, one residual scale per piece
     o.sf_sp = (j & 1) == 0 ? L.sf_sp + atom_pos(r, j >> 1) : -1;
     o.sf_res = L.sf_res + atom_pos(r, j);
@@ -281,8 +305,17 @@ __device__ __forceinline__ void store16(uint8_t *chunk, const Spot &o, uint32_t 
                                         uint32_t r0, uint32_t r1, uint32_t sc_res) {
   if (!DENSE) {
     *reinterpret_cast<uint32_t *>(chunk + o.sp) = kept;
-    if (UNIT == 2) chunk[o.meta] = (uint8_t)meta;
-    else *reinterpret_cast<uint16_t *>(chunk + o.meta) = (uint16_t)meta;
+    if (UNIT == 2) {
+      chunk[o.meta] = (uint8_t)meta;
+    } else if (UNIT == 1) {
+      *reinterpret_cast<uint16_t *>(chunk + o.meta) = (uint16_t)meta;
+    } else {
+#pragma unroll
+      for (int b = 0; b < 3; ++b) {
+        const int mb = o.mb + b;
+        chunk[o.meta + (mb >> 4) * 2048 + (mb & 15)] = (uint8_t)(meta >> (8 * b));
+      }
+    }
     if (o.sf_sp >= 0) chunk[o.sf_sp] = (uint8_t)sc_sp;
   }
   *reinterpret_cast<uint2 *>(chunk + o.res) = make_uint2(r0, r1);
@@ -308,7 +341,7 @@ __device__ __forceinline__ void process16(uint8_t *chunk, const Spot &o, float *
                            fmaxf(fabsf(e[4]), fabsf(e[5])), fmaxf(fabsf(e[6]), fabsf(e[7])), km);
         gmax = fmaxf(gmax, km);
       }
-    } else {
+    } else if (UNIT == 1) {
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         const float *e = v + 4 * g;
@@ -316,6 +349,17 @@ __device__ __forceinline__ void process16(uint8_t *chunk, const Spot &o, float *
         nib[g] = top2_of_4(fabsf(e[0]), fabsf(e[1]), fabsf(e[2]), fabsf(e[3]), km);
         gmax = fmaxf(gmax, km);
       }
+    } else {
+      // elements 4:8: nib[g] holds group g's keep mask (8 bits, four set); the group maximum
+      // is always kept, so the backbone block amax is the amax of all 16 values
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        float a[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = fabsf(v[8 * g + i]);
+        nib[g] = top4_of_8(a);
+      }
+      gmax = amax16(v, 0.f);
     }
     // ---- backbone block amax: 16 stored (NVFP4) = 2 lanes, 32 stored (MXFP4) = 4 lanes
     gmax = fmaxf(gmax, __shfl_xor_sync(kFull, gmax, 1));
@@ -342,6 +386,30 @@ __device__ __forceinline__ void process16(uint8_t *chunk, const Spot &o, float *
       w0 &= (0xFFu << (8 * (n0 & 3u))) | (0xFFu << (8 * (n0 >> 2)));
       w1 &= (0xFFu << (8 * (n1 & 3u))) | (0xFFu << (8 * (n1 >> 2)));
       meta = n0 | (n1 << 4);
+    } else if (UNIT == kPat48) {
+      // group g = word g: keep the four selected nibbles in index order (16 bits), zero the
+      // others; metadata: the four indices, 3 bits each, ascending (12 bits per group)
+      kept = 0u;
+      meta = 0u;
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        uint32_t &w = g == 0 ? w0 : w1;
+        const uint32_t keep = nib[g];
+        uint32_t q = 0u, m = 0u, nmask = 0u;
+        int pos = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if ((keep >> i) & 1u) {
+            q |= ((w >> (4 * i)) & 0xFu) << (4 * pos);
+            m |= (uint32_t)i << (3 * pos);
+            nmask |= 0xFu << (4 * i);
+            ++pos;
+          }
+        }
+        w &= nmask;
+        kept |= q << (16 * g);
+        meta |= m << (12 * g);
+      }
     } else {
       // group g = 16 bits (4 nibbles) of the words; kept nibbles i0, i1 -> one byte
       kept = 0u;
@@ -773,6 +841,8 @@ cudaError_t launch_prep(PrepParams p, int fmt, int unit, bool norm, bool dense, 
                        : launch_t<kFmtNV, 1, false, false, kSwiglu>(p, st);
     return unit == 2 ? launch_t<kFmtMX, 2, false, false, kSwiglu>(p, st) : launch_t<kFmtMX, 1, false, false, kSwiglu>(p, st);
   }
+  if (unit == kPat48)  // four of eight elements (sharq_prepare only)
+    return fmt == kFmtNV ? launch_n<kFmtNV, kPat48, false>(p, norm, st) : launch_n<kFmtMX, kPat48, false>(p, norm, st);
   if (fmt == kFmtNV)
     return unit == 2 ? launch_n<kFmtNV, 2, false>(p, norm, st) : launch_n<kFmtNV, 1, false>(p, norm, st);
   return unit == 2 ? launch_n<kFmtMX, 2, false>(p, norm, st) : launch_n<kFmtMX, 1, false>(p, norm, st);

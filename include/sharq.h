@@ -37,12 +37,15 @@
  * kept (key = largest |x| in the unit; equal keys go to the lower unit). The
  * sparse FP4 tensor-core MMA of sm_100a selects pairs, so the pattern
  * sharq_linear executes is (nm_n, nm_m, unit) = (2, 4, 2): two of every four
- * aligned pairs, i.e. 4 of 8 elements. sharq_prepare also computes the
- * element pattern (2, 4, 1).
+ * aligned pairs, i.e. 4 of 8 elements. sharq_prepare (and only it) also computes
+ * the element patterns (2, 4, 1) and (4, 8, 1), which no sparse FP4 MMA of sm_100a
+ * executes: sharq_linear rejects them with SHARQ_ERR_UNSUPPORTED.
  *
- * Sparse metadata. One 4-bit entry per group, the two kept unit indices
+ * Sparse metadata. 2:4: one 4-bit entry per group, the two kept unit indices
  * (i0 < i1) as i0 | i1<<2; group g of a row at bits 4g..4g+3 of that row's bit
  * string (per 256 K positions: 128 bits for pairs, 256 bits for elements).
+ * 4:8 over elements: one 12-bit entry per group of 8, the four kept indices
+ * ascending as i0 | i1<<3 | i2<<6 | i3<<9, group g at bits 12g..12g+11 (384 bits).
  *
  * Tiled operands. Activations and weights are stored as the tensor-core GEMM reads
  * them: chunks of 128 rows x 256 K positions, one contiguous chunk per (128-row block
@@ -60,10 +63,12 @@
  * Prepared activation chunk (sharq_prepare), B = 16 (NVFP4) or 32 (MXFP4):
  *   residual codes  offset 0,      128 rows x 128 bytes (256 codes)
  *   backbone codes  offset 16384,  128 rows x 64 bytes (the 128 kept codes, in K order)
- *   metadata        offset 24576,  2048 bytes (pairs) or 4096 bytes (elements)
+ *   metadata        offset 24576,  2048 bytes (pairs), 4096 (elements 2:4) or 6144
+ *                   (elements 4:8: byte b of row r's 48 at (b/16)*2048 + r*16 + b%16)
  *   backbone scales then residual scales, scale runs of 128/B and 256/B scales per row
- *   C = 29696 (NVFP4, pairs), 28672 (MXFP4, pairs), 31744 (NVFP4, elements),
- *       30720 (MXFP4, elements); padded rows: tokens_pad = tokens rounded up to 256.
+ *   C = 29696 (NVFP4, pairs), 28672 (MXFP4, pairs), 31744 (NVFP4, elements 2:4),
+ *       30720 (MXFP4, elements 2:4), 33792 (NVFP4, 4:8), 32768 (MXFP4, 4:8);
+ *       padded rows: tokens_pad = tokens rounded up to 256.
  * Dense-quantized activation chunk (sharq_quantize_dense): codes at 0 (128 x 128 bytes),
  *   scale run at 16384 (256/B scales per row); C = 18432 (NVFP4) or 17408 (MXFP4).
  * Packed weight chunk, for 128 weight rows = one half of a 256-row block (n_out_pad =
@@ -142,7 +147,7 @@ int sharq_pack_weight(const void *w_bf16_dev, int n_out, int k, int fmt, sharq_w
  *   x_bf16_dev      [tokens][k] row-major bf16 activations
  *   gamma_bf16_dev  [k] bf16 RMSNorm weight, or NULL for no normalization
  *   eps             RMSNorm epsilon (ignored without gamma)
- *   nm_n, nm_m, unit  the mask; (2,4,2) and (2,4,1) are executed
+ *   nm_n, nm_m, unit  the mask: (2,4,2), (2,4,1) or (4,8,1); only (2,4,2) feeds sharq_linear
  *   out             caller-filled struct of device buffers (shape fields are set here)
  * RMSNorm: rstd = 1/sqrt(fp32(sum(x^2)/k) + eps), xh = (x*rstd)*gamma in float32.
  * NVFP4 row scale s_x = amax|xh|/2688 (1 for a zero row), shared by backbone

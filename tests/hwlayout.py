@@ -4,7 +4,8 @@ Test infrastructure, written from the layout contract in include/sharq.h ("Tiled
 operands"), not from the CUDA sources: chunks of 128 rows x 256 K, chunk-major
 [row block][K step]; E2M1 pairs with the lower K index in the low nibble; code rows
 with their 16-byte units swizzled by row bits; scale runs of 128x4 atoms; metadata
-bit strings of 16 bytes per row per 256 K (pairs) or two such halves (elements).
+bit strings of 16 bytes per row per 256 K (pairs), two such halves (elements 2:4) or three
+(elements 4:8, 12-bit entries).
 """
 from __future__ import annotations
 
@@ -18,12 +19,13 @@ def to_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy()
 
 
-def act_layout(block: int, unit: int, sparse: bool = True) -> dict:
-    """Byte offsets inside one activation chunk and the chunk size C (header table)."""
+def act_layout(block: int, unit: int, sparse: bool = True, m: int = 4) -> dict:
+    """Byte offsets inside one activation chunk and the chunk size C (header table); m = 8
+    for the 4:8 element pattern."""
     sf_sp, sf_res = 128 // block, 256 // block  # scales per row per K step
     if not sparse:
         return dict(res=0, sf_res=16384, bytes=_round1k(16384 + 128 * sf_res), spk_res=sf_res)
-    meta = 2048 if unit == 2 else 4096
+    meta = 6144 if m == 8 else 2048 if unit == 2 else 4096
     off_sp = 24576 + meta
     off_res = off_sp + 128 * sf_sp
     return dict(res=0, sp=16384, meta=24576, sf_sp=off_sp, sf_res=off_res, bytes=_round1k(off_res + 128 * sf_res),
@@ -94,13 +96,35 @@ def meta_idx(buf: np.ndarray, tokens: int, k: int, unit: int, chunk: int, off: i
     return np.stack([nib & 3, nib >> 2], axis=-1).astype(np.int64)
 
 
+def meta_idx48(buf: np.ndarray, tokens: int, k: int, chunk: int, off: int) -> np.ndarray:
+    """Kept element indices [tokens, k/8, 4] of the 4:8 pattern: 12-bit entries (3 bits per
+    index, ascending), group g of a K step at bits 12g.. of the row's 48 bytes, byte b of
+    those at (b/16)*2048 + r*16 + b%16."""
+    b = np.asarray(buf, dtype=np.uint8).reshape(-1)
+    g = np.arange(k // 8)[None, :]
+    t = np.arange(tokens)[:, None]
+    ks, gg = g // 32, g % 32
+    base = _chunk_base(t, ks, k, chunk) + off + (t % 128) * 16
+    bit0 = 12 * gg
+    val = np.zeros(g.shape[:1] + (tokens, k // 8), dtype=np.int64)[0]
+    for d in range(3):  # the three bytes that can hold bits of the entry
+        byte = bit0 // 8 + d
+        byte_c = np.minimum(byte, 47)
+        addr = base + (byte_c // 16) * 2048 + byte_c % 16
+        val |= np.where(byte < 48, b[addr].astype(np.int64), 0) << (8 * d)
+    entry = (val >> (bit0 % 8)) & 0xFFF
+    return np.stack([(entry >> (3 * i)) & 7 for i in range(4)], axis=-1)
+
+
 def read_prep(p, block: int) -> dict:
-    """Canonical arrays of a library Prep (pattern 2:4) for comparison with oracle.prepare."""
+    """Canonical arrays of a library Prep (2:4 or 4:8) for comparison with oracle.prepare."""
     T, K, unit = p.tokens, p.k, p.unit
-    L = act_layout(block, unit)
+    m = getattr(p, "nm_m", 4)
+    L = act_layout(block, unit, m=m)
     buf = to_np(p.tiles)
     return dict(
-        idx=meta_idx(buf, T, K, unit, L["bytes"], L["meta"]),
+        idx=(meta_idx48(buf, T, K, L["bytes"], L["meta"]) if m == 8 else
+             meta_idx(buf, T, K, unit, L["bytes"], L["meta"])),
         sp_codes=nibbles(code_bytes(buf, T, K, L["bytes"], L["sp"], 64)),
         sp_scales=scale_run(buf, T, K, L["bytes"], L["sf_sp"], L["spk_sp"]),
         res_codes=nibbles(code_bytes(buf, T, K, L["bytes"], L["res"], 128)),

@@ -49,6 +49,12 @@ def test_prep_buffer_sizes(S):
     assert S.sharq_dense_buffer_sizes(T, K, "mxfp4") == [chunks * 17408, T * 4]
 
 
+def test_prep_buffer_sizes_4of8(S):
+    # four of eight elements: 48 metadata bytes per row per K step (6144 per chunk)
+    assert S.sharq_prep_buffer_sizes(300, 512, 4, 8, 1, "nvfp4") == [(512 // 128) * 2 * 33792, 1200]
+    assert S.sharq_prep_buffer_sizes(300, 512, 4, 8, 1, "mxfp4") == [(512 // 128) * 2 * 32768, 1200]
+
+
 def test_wpack_buffer_sizes(S):
     assert S.sharq_wpack_buffer_sizes(6144, 4096, "nvfp4") == [(6144 // 128) * 16 * 22528, 8]
     assert S.sharq_wpack_buffer_sizes(208, 256, "mxfp4") == [(256 // 128) * 1 * 19456, 8]
@@ -60,7 +66,8 @@ def test_wpack_buffer_sizes(S):
     ((16, 4096, 3, 2, 2, 0), 1),    # N > M
     ((16, 4096, 2, 4, 3, 0), 1),    # bad unit
     ((16, 4096, 2, 4, 2, 7), 1),    # bad format
-    ((16, 4096, 4, 8, 1, 0), 2),    # valid pattern this build does not execute
+    ((16, 4096, 1, 4, 2, 0), 2),    # valid pattern this build does not compute
+    ((16, 4096, 4, 8, 2, 0), 2),    # 4:8 over pairs: not computed (4:8 is over elements)
 ])
 def test_prep_sizes_reject(S, args, status):
     sizes = (ctypes.c_size_t * 2)()
@@ -78,7 +85,7 @@ def test_calls_reject_bad_arguments_before_launch(S):
     assert S.lib.sharq_prepare(ctypes.c_void_p(0x1008), 16, 4096, None, 1e-6, 2, 4, 2, 0, ctypes.byref(P),
                                null) == S.SHARQ_ERR_INVALID_ARG
     # unsupported pattern
-    assert S.lib.sharq_prepare(ctypes.c_void_p(0x1000), 16, 4096, None, 1e-6, 4, 8, 1, 0, ctypes.byref(P),
+    assert S.lib.sharq_prepare(ctypes.c_void_p(0x1000), 16, 4096, None, 1e-6, 1, 4, 2, 0, ctypes.byref(P),
                                null) == S.SHARQ_ERR_UNSUPPORTED
     # null output buffers in the struct
     assert S.lib.sharq_prepare(ctypes.c_void_p(0x1000), 16, 4096, None, 1e-6, 2, 4, 2, 0, ctypes.byref(P),
