@@ -502,6 +502,8 @@ def run_sharq(args, rank, world, local):
         del w0
         ps = [S.alloc_prep(T_, K_, 2, 4, 2, fmt) for _ in range(n)]
         ys_ = [torch.empty(T_, N_, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+        ws_bytes = S.sharq_linear_workspace_size(T_, N_, K_)  # split K where few tiles
+        ws_ = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda") if ws_bytes else None
 
         def prep_all(st):
             for i in range(n):
@@ -509,12 +511,12 @@ def run_sharq(args, rank, world, local):
 
         def lin_all(st):
             for i in range(n):
-                S.sharq_linear(ps[i], wps_[i], y=ys_[i], stream=st)
+                S.sharq_linear(ps[i], wps_[i], y=ys_[i], stream=st, workspace=ws_)
 
         def step_all(st):
             for i in range(n):
                 S.sharq_prepare(xs_[i], g_, 1e-6, 2, 4, 2, fmt, out=ps[i], stream=st)
-                S.sharq_linear(ps[i], wps_[i], y=ys_[i], stream=st)
+                S.sharq_linear(ps[i], wps_[i], y=ys_[i], stream=st, workspace=ws_)
 
         step_all(stream)
         torch.cuda.synchronize()
@@ -526,7 +528,8 @@ def run_sharq(args, rank, world, local):
                 "tokens_per_s": T_ / (ts / 1e3), "eff_fp4_tflops": 2.0 * T_ * N_ * K_ / (ts / 1e3) / 1e12,
                 "gemm_tflops": gt, "gemm_frac": gt / fp4_peak[fmt],
                 "prep_gbs": pb / (tp / 1e3) / 1e9, "prep_frac": pb / (tp / 1e3) / 1e9 / hbm_peak,
-                "l2": f"{n} rotating set(s)"}
+                "split_k": ws_bytes // (4 * T_ * N_) if ws_bytes else 1,
+                "w_gbs": N_ * K_ * 0.5625 / (tl / 1e3) / 1e9, "l2": f"{n} rotating set(s)"}
 
     def measure_prep_only(name, T_, K_, fmt, nm, seed):
         """A mask pattern no sparse FP4 MMA executes (elements 2:4, elements 4:8): the

@@ -71,6 +71,8 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sharq_tensor_scale_workspace_size": (S, [I, I]),
         "sharq_prepare_tensor_scale": (I, [P, I, I, P, F, I, I, I, I, ctypes.POINTER(_Prep), P, P]),
         "sharq_linear": (I, [ctypes.POINTER(_Prep), ctypes.POINTER(_WPack), P, I, P]),
+        "sharq_linear_workspace_size": (S, [I, I, I]),
+        "sharq_linear_split": (I, [ctypes.POINTER(_Prep), ctypes.POINTER(_WPack), P, I, P, S, P]),
         "sharq_linear_grouped": (I, [ctypes.POINTER(_Prep), ctypes.POINTER(_WPack), ctypes.POINTER(P), I, I, P]),
         "sharq_quantize_dense": (I, [P, I, I, P, F, I, P, P, P]),
         "sharq_linear_dense": (I, [P, P, I, I, ctypes.POINTER(_WPack), P, I, P]),
@@ -287,13 +289,25 @@ def sharq_prepare_swiglu(gate_up: torch.Tensor, nm_n: int = 2, nm_m: int = 4, un
 
 
 def sharq_linear(prep: Prep, w: WPack, y: torch.Tensor | None = None, out_dtype=torch.bfloat16,
-                 stream=None) -> torch.Tensor:
-    """Y [tokens, n_out] = sparse FP4 GEMM (backbone) + dense FP4 GEMM (residual), one output."""
+                 stream=None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Y [tokens, n_out] = sparse FP4 GEMM (backbone) + dense FP4 GEMM (residual), one output.
+    With `workspace` (device bytes, sharq_linear_workspace_size) the split-K form runs where the
+    shape calls for it (sharq_linear_split)."""
     if y is None:
         y = torch.empty(prep.tokens, w.n_out, dtype=out_dtype, device=prep.tiles.device)
     code = SHARQ_OUT_F32 if y.dtype == torch.float32 else SHARQ_OUT_BF16
-    _check(lib.sharq_linear(ctypes.byref(prep.struct()), ctypes.byref(w.struct()), _ptr(y), code, _stream(stream)))
+    if workspace is not None:
+        _check(lib.sharq_linear_split(ctypes.byref(prep.struct()), ctypes.byref(w.struct()), _ptr(y), code,
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    else:
+        _check(lib.sharq_linear(ctypes.byref(prep.struct()), ctypes.byref(w.struct()), _ptr(y), code,
+                                _stream(stream)))
     return y
+
+
+def sharq_linear_workspace_size(tokens: int, n_out: int, k: int) -> int:
+    """Bytes of workspace the split-K form of sharq_linear wants for this shape (0: none)."""
+    return int(lib.sharq_linear_workspace_size(tokens, n_out, k))
 
 
 def sharq_linear_grouped(preps: list[Prep], ws: list[WPack], ys: list[torch.Tensor] | None = None,

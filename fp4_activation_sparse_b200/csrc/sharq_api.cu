@@ -337,6 +337,49 @@ int sharq_linear(const sharq_prep *a, const sharq_wpack *w, void *y, int out_dty
   return run_gemm(g, "sharq_linear", static_cast<cudaStream_t>(stream));
 }
 
+size_t sharq_linear_workspace_size(int tokens, int n_out, int k) {
+  if (check_shape(tokens, k, "tokens")) return 0;
+  if (n_out < 16 || n_out % 16) { fail(SHARQ_ERR_INVALID_ARG, "n_out must be a positive multiple of 16"); return 0; }
+  const int S = sharq::gemm_split_count(tokens, n_out, k);
+  g_err[0] = 0;
+  return S > 1 ? (size_t)S * tokens * n_out * sizeof(float) : 0;
+}
+
+int sharq_linear_split(const sharq_prep *a, const sharq_wpack *w, void *y, int out_dtype, void *workspace,
+                       size_t workspace_bytes, void *stream) {
+  if (int s = check_linear(a, w, y, out_dtype)) return s;
+  const int S = sharq::gemm_split_count(a->tokens, w->n_out, a->k);
+  if (S <= 1) return sharq_linear(a, w, y, out_dtype, stream);
+  const size_t plane = (size_t)a->tokens * w->n_out;
+  const size_t need = (size_t)S * plane * sizeof(float);
+  if (!workspace || workspace_bytes < need)
+    return fail(SHARQ_ERR_INVALID_ARG, "sharq_linear_split: this launch needs a workspace of %zu bytes (got %zu)",
+                need, workspace ? workspace_bytes : (size_t)0);
+  if (!aligned16(workspace)) return fail(SHARQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  sharq::GemmParams g;
+  memset(&g, 0, sizeof g);
+  const int ks = a->k / 256, q = (ks + S - 1) / S;
+  for (int s = 0; s < S; ++s) {
+    set_group(g.grp[s], a->tiles, a->row_scale, a->tokens, w, static_cast<float *>(workspace) + s * plane);
+    g.grp[s].k0 = s * q;
+    g.grp[s].num_k = ks - s * q < q ? ks - s * q : q;
+  }
+  g.n_groups = S;
+  g.N = w->n_out;
+  g.K = a->k;
+  g.N_pad = sharq::round_up(w->n_out, 256);
+  g.fmt = a->fmt;
+  g.out_f32 = 1;  // partial outputs
+  g.sparse = 1;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (int s = run_gemm(g, "sharq_linear_split", st)) return s;
+  cudaError_t e = sharq::launch_splitk_reduce(static_cast<const float *>(workspace), S, a->tokens, w->n_out, y,
+                                              out_dtype == SHARQ_OUT_F32, st);
+  if (e != cudaSuccess) return cuda_fail(e, "sharq_linear_split (reduction)");
+  g_err[0] = 0;
+  return SHARQ_OK;
+}
+
 int sharq_linear_grouped(const sharq_prep *a, const sharq_wpack *w, void *const *y, int n_groups, int out_dtype,
                          void *stream) {
   if (!a || !w || !y) return fail(SHARQ_ERR_INVALID_ARG, "null group arrays");

@@ -397,7 +397,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   using L = Stage<MX, SPARSE>;
   constexpr int apt_res = atoms_res(MX ? 1 : 0), apt_sp = atoms_sp(MX ? 1 : 0);
   constexpr int kStageBytes = L::kBytes;
-  const int num_k = p.K / BK;
+  const int ks_total = p.K / BK;  // K steps per operand row block: the chunk stride
   const int num_tiles = p.num_tiles;
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
   const uint64_t limit = p.wait_limit > 0 ? (uint64_t)p.wait_limit : 4000000000ull;
@@ -432,8 +432,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // The packed weight is not an output of the preparation: its first K steps for this CTA's
     // first tile are fetched into L2 while the preparation may still be running.
     const int g = group_of<MAXG>(p, pair), lt = pair - p.grp[g].tile_begin;
-    const int w_row0 = ((lt / p.grp[g].num_m) * BN / 128 + (int)rank) * num_k * (L::W.bytes / 1024);
-    for (int kt = 0; kt < kStages && kt < num_k; ++kt) tma_prefetch_l2(&ms.m[g].w, 0, w_row0 + kt * (L::W.bytes / 1024));
+    const int w_row0 = (((lt / p.grp[g].num_m) * BN / 128 + (int)rank) * ks_total + p.grp[g].k0) * (L::W.bytes / 1024);
+    for (int kt = 0; kt < kStages && kt < p.grp[g].num_k; ++kt)
+      tma_prefetch_l2(&ms.m[g].w, 0, w_row0 + kt * (L::W.bytes / 1024));
   }
   // Launched as a programmatic dependent of the preparation: the prologue above overlaps its
   // tail; its outputs are read only after it has completed and flushed.
@@ -452,8 +453,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const TmaMaps &maps = ms.m[g];
         const int m0 = (lt % num_m) * (2 * BM) + (int)rank * BM;  // this CTA's activation rows
         const int n0 = (lt / num_m) * BN;                          // the pair's output columns
-        const int a_row0 = (m0 / 128) * num_k * (L::A.bytes / 1024);  // chunk rows of 1024 bytes
-        const int w_row0 = (n0 / 128 + (int)rank) * num_k * (L::W.bytes / 1024);
+        // chunk rows of 1024 bytes; the group's K steps start at k0
+        const int a_row0 = ((m0 / 128) * ks_total + p.grp[g].k0) * (L::A.bytes / 1024);
+        const int w_row0 = ((n0 / 128 + (int)rank) * ks_total + p.grp[g].k0) * (L::W.bytes / 1024);
+        const int num_k = p.grp[g].num_k;
         for (int kt = 0; kt < num_k; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, limit, abort_flag)) { ok = false; break; }
           const uint32_t st = smem0 + stage * kStageBytes;
@@ -488,6 +491,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // released by both CTAs' epilogue warps (remote arrives): cluster-scope acquire
         if (!mbar_wait<true>(acc_empty, acc_phase ^ 1u, limit, abort_flag)) { ok = false; break; }
         tc_fence_after();
+        const int num_k = p.grp[group_of<MAXG>(p, tile)].num_k;
         for (int kt = 0; kt < num_k; ++kt) {
           // the scale writers of both CTAs waited for their stage's bytes, then wrote its scales
           // (remote arrives: cluster-scope acquire)
@@ -664,6 +668,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t phase = 0, buf = 0, buf_phase = 0;
     bool ok = true;
     for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+      const int num_k = p.grp[group_of<MAXG>(p, tile)].num_k;
       for (int kt = 0; kt < num_k; ++kt) {
         if (!mbar_wait_warp(full_bar(stage), phase, limit, abort_flag)) { ok = false; break; }
         // the buffer is free once the MMAs that last read it (kScaleBufs steps ago) completed
@@ -1008,12 +1013,88 @@ cudaError_t launch_gemm(GemmParams p, cudaStream_t st, const char **why) {
   int tiles = 0;
   const int num_n = (p.N + BN - 1) / BN;
   for (int g = 0; g < p.n_groups; ++g) {
+    if (p.grp[g].num_k == 0) p.grp[g].num_k = p.K / BK - p.grp[g].k0;
     p.grp[g].num_m = (p.grp[g].T + 2 * BM - 1) / (2 * BM);
     p.grp[g].tile_begin = tiles;
     tiles += p.grp[g].num_m * num_n;
   }
   p.num_tiles = tiles;
   return p.n_groups == 1 ? launch_groups<1>(p, st, why) : launch_groups<kMaxGroups>(p, st, why);
+}
+
+// ---------------------------------------------------------------- split K
+// A launch with few output tiles leaves most SM pairs idle; its K range is then cut into S
+// slices, run as S groups of one grouped launch that write float32 partial outputs (each
+// already scaled by s_x * s_w), and summed in slice order by a second kernel.
+int sm_count() {
+  static std::once_flag once[kMaxDevices];
+  static int sms[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::call_once(once[dev], [dev] {
+    if (cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms[dev] = 0;
+  });
+  return sms[dev];
+}
+
+// Slices for a (tokens x n_out x k) linear, from a cost estimate: a pair spends about 0.5 us
+// per K step of a tile (the tensor pipe's rate at these tile sizes), so one slice of q steps
+// saves (K steps - q) * 0.5 us when every pair holds at most one tile; the split form costs a
+// second launch (~3 us) and the float32 partials written and read back (S * tokens * n_out *
+// 8 bytes at ~3 TB/s, L2-resident). 1 when the tiles already fill half of the SM pairs or
+// slicing does not pay; at most kMaxGroups slices, at least 2 K steps each.
+int gemm_split_count(int tokens, int n_out, int k) {
+  const int pairs = sm_count() / 2;
+  const int tiles = ((tokens + 2 * BM - 1) / (2 * BM)) * ((n_out + BN - 1) / BN);
+  const int ks = k / BK;
+  if (pairs < 2 || 2 * tiles > pairs) return 1;
+  int s_max = pairs / tiles;
+  if (s_max > kMaxGroups) s_max = kMaxGroups;
+  if (s_max > ks / 2) s_max = ks / 2;
+  double best = 0.5 * ks;
+  int best_s = 1;
+  for (int S = 2; S <= s_max; ++S) {
+    const int q = (ks + S - 1) / S;
+    const double est = 0.5 * q + 3.0 + (double)S * tokens * n_out * 8.0 / 3.0e6;
+    if (est < best) {
+      best = est;
+      best_s = (ks + q - 1) / q;  // every slice non-empty
+    }
+  }
+  return best_s;
+}
+
+namespace {
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4 *ws, int S, long long n4, long long plane4,
+                                                            void *y, int out_f32) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    float4 a = __ldcs(ws + i);
+    for (int s = 1; s < S; ++s) {  // slice order: a fixed summation order
+      const float4 b = __ldcs(ws + s * plane4 + i);
+      a.x = __fadd_rn(a.x, b.x);
+      a.y = __fadd_rn(a.y, b.y);
+      a.z = __fadd_rn(a.z, b.z);
+      a.w = __fadd_rn(a.w, b.w);
+    }
+    if (out_f32) {
+      reinterpret_cast<float4 *>(y)[i] = a;
+    } else {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+      reinterpret_cast<uint2 *>(y)[i] =
+          make_uint2(*reinterpret_cast<const uint32_t *>(&lo), *reinterpret_cast<const uint32_t *>(&hi));
+    }
+  }
+}
+}  // namespace
+
+cudaError_t launch_splitk_reduce(const float *ws, int S, int T, int N, void *y, int out_f32, cudaStream_t st) {
+  const long long n4 = (long long)T * N / 4;  // N is a multiple of 16
+  long long blocks = (n4 + 255) / 256;
+  const long long cap = 8ll * (sm_count() > 0 ? sm_count() : 148);
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(ws), S, n4, n4, y, out_f32);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_mma_peak(int mode, int fmt, int iters, int clusters, cudaStream_t st) {

@@ -78,6 +78,8 @@ struct GemmGroup {
   void *y;                    // [T][N]
   int T, T_pad;
   int tile_begin, num_m;      // first pair tile of this group in the launch, its 256-row blocks
+  int k0, num_k;              // the group's K steps (of 256): k0 .. k0 + num_k - 1 (split K);
+                              // num_k = 0 means all of K
 };
 
 constexpr int kMaxGroups = 32;  // groups per launch of the grouped GEMM
@@ -101,6 +103,9 @@ cudaError_t launch_pack(PackParams p, int fmt, cudaStream_t st);
 cudaError_t launch_gemm(GemmParams p, cudaStream_t st, const char **why);
 cudaError_t read_and_clear_device_status(int *status, cudaStream_t st);
 cudaError_t launch_mma_peak(int mode, int fmt, int iters, int clusters, cudaStream_t st);
+int sm_count();
+int gemm_split_count(int tokens, int n_out, int k);
+cudaError_t launch_splitk_reduce(const float *ws, int S, int T, int N, void *y, int out_f32, cudaStream_t st);
 cudaError_t launch_rmsnorm(const uint16_t *x, const uint16_t *gamma, float eps, int T, int K, uint16_t *y,
                            cudaStream_t st);
 

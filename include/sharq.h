@@ -227,6 +227,22 @@ int sharq_prepare_swiglu(const void *gate_up_bf16_dev, int tokens, int k, int nm
 int sharq_linear(const sharq_prep *a, const sharq_wpack *w, void *y_dev, int out_dtype,
                  void *stream);
 
+/* sharq_linear for launches with few output tiles (few tokens and a narrow output), where a
+ * plain launch leaves most SM pairs idle while one pair walks all of K: with a caller
+ * workspace the K range is cut into S slices (S from sharq_linear_workspace_size's shape
+ * rule), run as S problems of one grouped launch that each write float32 partial outputs
+ * already scaled by s_x * s_w, then summed in slice order by a second kernel into y (bf16
+ * rounded once, at the end). The same two MMA paths and scales as sharq_linear; the result
+ * differs from it only by float32 rounding order. When the shape does not call for slicing,
+ * this is exactly sharq_linear and the workspace is not touched.
+ *   workspace_dev    device buffer of at least sharq_linear_workspace_size(tokens, n_out, k)
+ *                    bytes, 16-byte aligned, contents irrelevant; overwritten. Calls whose
+ *                    launches may overlap on the GPU need distinct workspaces.
+ * Errors as sharq_linear; SHARQ_ERR_INVALID_ARG if the workspace is smaller than needed. */
+size_t sharq_linear_workspace_size(int tokens, int n_out, int k);
+int sharq_linear_split(const sharq_prep *a, const sharq_wpack *w, void *y_dev, int out_dtype,
+                       void *workspace_dev, size_t workspace_bytes, void *stream);
+
 /* Grouped (mixture-of-experts) SharQ linear: n_groups independent problems
  * Y_e = sharq_linear(a[e], w[e]) computed by one launch per 32 groups, the CTA pairs working
  * through the output tiles of all groups (each expert's tokens prepared by sharq_prepare into
