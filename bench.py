@@ -470,7 +470,7 @@ def run_sharq(args, rank, world, local):
     moe_tflops = moe_work / (t_moe_gemm / 1e3) / 1e12
     moe_line = {"workload": f"qwen3_30b_a3b experts gate_up T={T} top-{moe['top_k']} of {E}, K={Km} N={Nm} nvfp4",
                 "routed_rows": int(counts.sum()), "padded_rows": rows_pad, "launches": "1 prep + "
-                f"{(E + 31) // 32} grouped GEMM", "t_prep_us": t_moe_prep * 1e3, "t_grouped_gemm_us": t_moe_gemm * 1e3,
+                f"{(E + 63) // 64} grouped GEMM", "t_prep_us": t_moe_prep * 1e3, "t_grouped_gemm_us": t_moe_gemm * 1e3,
                 "achieved_tflops": moe_tflops, "peak_tflops": fp4_peak["nvfp4"],
                 "frac": moe_tflops / fp4_peak["nvfp4"]}
     del x_moe, x_moe_tok, wps_moe, p_moe, views, ys_moe

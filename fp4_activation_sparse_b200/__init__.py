@@ -313,7 +313,7 @@ def sharq_linear_workspace_size(tokens: int, n_out: int, k: int) -> int:
 def sharq_linear_grouped(preps: list[Prep], ws: list[WPack], ys: list[torch.Tensor] | None = None,
                          out_dtype=torch.bfloat16, stream=None) -> list[torch.Tensor]:
     """Mixture-of-experts form: Y_e = sharq_linear(preps[e], ws[e]) for every expert in one
-    launch (per 32 experts). Every weight shares n_out and k."""
+    launch (per 64 experts). Every weight shares n_out and k."""
     n = len(preps)
     assert n == len(ws) and n >= 1
     if ys is None:

@@ -371,6 +371,7 @@ template <int MAXG>
 struct __align__(64) TmaMapSet {
   TmaMaps m[MAXG];
 };
+static_assert(sizeof(TmaMapSet<kMaxGroups>) + sizeof(GemmParams) <= 32764, "kernel parameter space");
 
 // MAXG: 1 for one problem per launch, kMaxGroups for the grouped (mixture-of-experts) form.
 template <bool MX, bool SPARSE, int MAXG>

@@ -82,7 +82,9 @@ struct GemmGroup {
                               // num_k = 0 means all of K
 };
 
-constexpr int kMaxGroups = 32;  // groups per launch of the grouped GEMM
+// groups per launch of the grouped GEMM: its tensor maps (3 x 128 B per group) and group table
+// travel in the kernel parameters, which hold up to 32764 bytes
+constexpr int kMaxGroups = 64;
 
 struct GemmParams {
   GemmGroup grp[kMaxGroups];

@@ -244,7 +244,7 @@ int sharq_linear_split(const sharq_prep *a, const sharq_wpack *w, void *y_dev, i
                        void *workspace_dev, size_t workspace_bytes, void *stream);
 
 /* Grouped (mixture-of-experts) SharQ linear: n_groups independent problems
- * Y_e = sharq_linear(a[e], w[e]) computed by one launch per 32 groups, the CTA pairs working
+ * Y_e = sharq_linear(a[e], w[e]) computed by one launch per 64 groups, the CTA pairs working
  * through the output tiles of all groups (each expert's tokens prepared by sharq_prepare into
  * their own buffers, so no tile mixes experts). The abstract evaluates a mixture-of-experts
  * model (Qwen3-30B-A3B) with the method; this is its expert layer.
