@@ -60,7 +60,8 @@ namespace {
 constexpr int BM = 128;   // activation rows per CTA (256 per pair)
 constexpr int BN = 256;   // output columns per pair tile
 constexpr int BK = 256;   // logical K per stage
-constexpr int kStages = 4;
+constexpr int kStagesPair = 4;  // pipeline stages of the pair form
+constexpr int kStages1 = 3;     // of the single-CTA form (larger stages: both weight halves)
 constexpr int kEpiWarps = 8;
 constexpr int kSfWarps = 4;  // one per tensor-memory lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps + 32 * kSfWarps;  // producer, MMA, epilogue, scale writers
@@ -86,12 +87,21 @@ constexpr int kMaxStageBytes = 52224;  // NVFP4 SharQ: 29696 + 22528
 // rows x 32 columns (64-byte rows, 64-byte swizzle), reused four times per tile (on a pair's
 // last tile the boxes go to the then idle pipeline stages instead, four per warp)
 constexpr int kStageOutBytes = 2048;
-constexpr int kOutOffset = kStages * kMaxStageBytes;  // 1024-aligned
-constexpr int kSmemBytes = kOutOffset + kEpiWarps * kStageOutBytes + 1024 /*align slack*/ + 256 /*barriers*/;
+constexpr int kOutOffsetPair = kStagesPair * kMaxStageBytes;  // 1024-aligned
+constexpr int kSmemBytes = kOutOffsetPair + kEpiWarps * kStageOutBytes + 1024 /*align slack*/ + 256 /*barriers*/;
 static_assert(Stage<false, true>::kBytes <= kMaxStageBytes && Stage<true, true>::kBytes <= kMaxStageBytes, "stage");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-static_assert(kOutOffset % 1024 == 0, "staging alignment");
-static_assert(4 * kEpiWarps * kStageOutBytes <= kOutOffset, "last-tile boxes fit in the pipeline stages");
+static_assert(kOutOffsetPair % 1024 == 0, "staging alignment");
+static_assert(4 * kEpiWarps * kStageOutBytes <= kOutOffsetPair, "last-tile boxes fit in the pipeline stages");
+// single-CTA form: a stage adds the other weight half's codes (128 rows x 128 bytes)
+constexpr int kWCodeBytes = 16384;
+constexpr int kMaxStage1Bytes = 52224 + kWCodeBytes;
+constexpr int kOutOffset1 = kStages1 * kMaxStage1Bytes;
+constexpr int kSmemBytes1 = kOutOffset1 + kEpiWarps * kStageOutBytes + 1024 + 256;
+static_assert(Stage<false, true>::kBytes + kWCodeBytes <= kMaxStage1Bytes &&
+                  Stage<true, true>::kBytes + kWCodeBytes <= kMaxStage1Bytes, "single-CTA stage");
+static_assert(kSmemBytes1 <= 227 * 1024, "shared memory (single CTA)");
+static_assert(kOutOffset1 % 1024 == 0 && 4 * kEpiWarps * kStageOutBytes <= kOutOffset1, "single-CTA staging");
 
 struct __align__(64) TmaMaps {
   CUtensorMap act, w;  // both: rows of 1024 bytes (256 x u32), one box = one chunk
@@ -215,6 +225,54 @@ __device__ __forceinline__ void tc_commit_both(uint32_t bar) {
       : "memory");
 }
 
+// commit to this CTA's barrier only (single-CTA form)
+__device__ __forceinline__ void tc_commit_own(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+template <bool PAIR>
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  if (PAIR) tc_commit_both(bar);
+  else tc_commit_own(bar);
+}
+
+template <bool PAIR>
+__device__ __forceinline__ void tmem_alloc(uint32_t slot) {
+  if (PAIR) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  } else {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+}
+template <bool PAIR>
+__device__ __forceinline__ void tmem_dealloc(uint32_t tmem) {
+  if (PAIR) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  else asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+}
+// the pair's CTAs, or this CTA's threads
+template <bool PAIR>
+__device__ __forceinline__ void block_sync() {
+  if (PAIR) cluster_sync();
+  else __syncthreads();
+}
+
+// 2-D TMA load into this CTA's shared memory (single-CTA form: no cta_group qualifier)
+__device__ __forceinline__ void tma_load_2d_1cta(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+// contiguous bytes from global into this CTA's shared memory (both 16-byte aligned, a multiple of
+// 16 bytes), completing on `bar`
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 // L2 prefetch of the 2-D box at (c0, c1) of a tensor map (no shared memory, no completion)
 __device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap *map, int c0, int c1) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(c0), "r"(c1)
@@ -246,7 +304,8 @@ __device__ __forceinline__ uint64_t dsc(uint64_t tmpl, uint32_t addr16) { return
 
 // Instruction descriptor of the block-scaled MMA kinds (mxf4 / mxf4nvf4): E2M1 A and B,
 // K-major, fp32 accumulate, M = 256 (two CTAs), N = 256.
-__device__ __forceinline__ uint32_t idesc_bs(bool sparse, bool ue8m0, uint32_t sfa_id, uint32_t sfb_id) {
+__device__ __forceinline__ uint32_t idesc_bs(bool sparse, bool ue8m0, uint32_t sfa_id, uint32_t sfb_id,
+                                             bool pair = true) {
   uint32_t d = 0;
   d |= (sparse ? 1u : 0u) << 2;
   d |= (sfb_id & 3u) << 4;
@@ -254,43 +313,48 @@ __device__ __forceinline__ uint32_t idesc_bs(bool sparse, bool ue8m0, uint32_t s
   d |= 1u << 10;                         // B format E2M1
   d |= (uint32_t)(BN >> 3) << 17;        // N
   d |= (ue8m0 ? 1u : 0u) << 23;          // scale type: 0 UE4M3, 1 UE8M0
-  d |= (uint32_t)((2 * BM) >> 4) << 24;  // M
+  d |= (uint32_t)((pair ? 2 * BM : BM) >> 4) << 24;  // M: 256 over the pair, or 128 on one CTA
   d |= (sfa_id & 3u) << 29;
   return d;
 }
 
-template <bool MX>
+// Block-scaled FP4 MMAs, dense and structured-sparse, on the CTA pair (cta_group::2, M = 256)
+// or on one CTA (cta_group::1, M = 128). The kind and block size follow the format.
+#define SHARQ_MMA_DENSE(CG, KIND)                                                                              \
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"                                            \
+               "tcgen05.mma.cta_group::" CG ".kind::" KIND " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem), \
+               "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb))
+#define SHARQ_MMA_SPARSE(CG, KIND)                                                                           \
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"                                          \
+               "tcgen05.mma.sp.cta_group::" CG ".kind::" KIND " [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}" ::"r"( \
+                   d_tmem),                                                                                  \
+               "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb), "r"(meta))
+
+template <bool MX, bool PAIR = true>
 __device__ __forceinline__ void mma_dense(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
                                           uint32_t sfb, uint32_t acc) {
-  if (MX)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
-            d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
+  if (PAIR) {
+    if (MX) SHARQ_MMA_DENSE("2", "mxf4.block_scale.block32");
+    else SHARQ_MMA_DENSE("2", "mxf4nvf4.block_scale.block16");
+  } else {
+    if (MX) SHARQ_MMA_DENSE("1", "mxf4.block_scale.block32");
+    else SHARQ_MMA_DENSE("1", "mxf4nvf4.block_scale.block16");
+  }
 }
 
-template <bool MX>
+template <bool MX, bool PAIR = true>
 __device__ __forceinline__ void mma_sparse(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t meta, uint32_t idesc,
                                            uint32_t sfa, uint32_t sfb, uint32_t acc) {
-  if (MX)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.sp.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}" ::"r"(
-            d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb), "r"(meta));
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.sp.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}" ::"r"(
-            d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb), "r"(meta));
+  if (PAIR) {
+    if (MX) SHARQ_MMA_SPARSE("2", "mxf4.block_scale.block32");
+    else SHARQ_MMA_SPARSE("2", "mxf4nvf4.block_scale.block16");
+  } else {
+    if (MX) SHARQ_MMA_SPARSE("1", "mxf4.block_scale.block32");
+    else SHARQ_MMA_SPARSE("1", "mxf4nvf4.block_scale.block16");
+  }
 }
+#undef SHARQ_MMA_DENSE
+#undef SHARQ_MMA_SPARSE
 
 // 32 lanes x 32 columns of 32 bits; asynchronous until tmem_ld_wait()
 __device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t *r) {
@@ -374,9 +438,12 @@ struct __align__(64) TmaMapSet {
 static_assert(sizeof(TmaMapSet<kMaxGroups>) + sizeof(GemmParams) <= 32764, "kernel parameter space");
 
 // MAXG: 1 for one problem per launch, kMaxGroups for the grouped (mixture-of-experts) form.
-template <bool MX, bool SPARSE, int MAXG>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    sharq_gemm_kernel(const __grid_constant__ TmaMapSet<MAXG> ms, const __grid_constant__ GemmParams p) {
+// PAIR: the CTA-pair form (cta_group::2, 256 x 256 tiles); otherwise one CTA per 128 x 256
+// tile (cta_group::1), for launches whose row groups are mostly at most 128 rows.
+template <bool MX, bool SPARSE, int MAXG, bool PAIR>
+__device__ __forceinline__ void gemm_body(const TmaMapSet<MAXG> &ms, const GemmParams &p) {
+  constexpr int kStages = PAIR ? kStagesPair : kStages1;
+  constexpr int kOutOffset = PAIR ? kOutOffsetPair : kOutOffset1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOutOffset + kEpiWarps * kStageOutBytes);
@@ -385,7 +452,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   volatile uint32_t *abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
   const bool leader = rank == 0;
   const uint32_t smem0 = smem_u32(smem);
   const uint32_t bar0 = smem_u32(bars);
@@ -397,10 +464,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   using L = Stage<MX, SPARSE>;
   constexpr int apt_res = atoms_res(MX ? 1 : 0), apt_sp = atoms_sp(MX ? 1 : 0);
-  constexpr int kStageBytes = L::kBytes;
+  // single-CTA stage: activation chunk, the two weight halves' codes back to back (one 256-row
+  // B operand), then the weight scales (both halves' atoms, as the pair form's chunk has them)
+  constexpr int kStageBytes = PAIR ? L::kBytes : L::kBytes + kWCodeBytes;
+  constexpr int kWScales = PAIR ? L::kW : L::kW + kWCodeBytes;  // the weight scale region's base
   const int ks_total = p.K / BK;  // K steps per operand row block: the chunk stride
   const int num_tiles = p.num_tiles;
-  const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+  // work units: CTA pairs, or single CTAs
+  const int pair = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int num_pairs = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const uint64_t limit = p.wait_limit > 0 ? (uint64_t)p.wait_limit : 4000000000ull;
 
   if (threadIdx.x == 0) {
@@ -409,9 +481,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(empty_bar(s), 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 2 * kEpiWarps);
+    mbar_init(acc_empty, (PAIR ? 2 : 1) * kEpiWarps);
     mbar_init(drain_bar, 1);
-    for (int s = 0; s < kStages; ++s) mbar_init(sf_full_bar(s), 2 * kSfWarps);  // writers of both CTAs
+    for (int s = 0; s < kStages; ++s) mbar_init(sf_full_bar(s), (PAIR ? 2 : 1) * kSfWarps);  // writers of both CTAs
     for (uint32_t b = 0; b < kScaleBufs; ++b) mbar_init(sf_free_bar(b), 1);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -420,22 +492,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(&ms.m[0].act) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&ms.m[0].w) : "memory");
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
-  }
+  if (warp == 1) tmem_alloc<PAIR>(smem_u32(tmem_slot));
   tc_fence_before();
-  cluster_sync();  // barriers initialized and TMEM allocated in both CTAs
+  block_sync<PAIR>();  // barriers initialized and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (warp == 0 && lane == 0 && pair < num_tiles) {
     // The packed weight is not an output of the preparation: its first K steps for this CTA's
     // first tile are fetched into L2 while the preparation may still be running.
     const int g = group_of<MAXG>(p, pair), lt = pair - p.grp[g].tile_begin;
-    const int w_row0 = (((lt / p.grp[g].num_m) * BN / 128 + (int)rank) * ks_total + p.grp[g].k0) * (L::W.bytes / 1024);
-    for (int kt = 0; kt < kStages && kt < p.grp[g].num_k; ++kt)
-      tma_prefetch_l2(&ms.m[g].w, 0, w_row0 + kt * (L::W.bytes / 1024));
+    for (int h = 0; h < (PAIR ? 1 : 2); ++h) {
+      const int w_row0 =
+          (((lt / p.grp[g].num_m) * BN / 128 + (PAIR ? (int)rank : h)) * ks_total + p.grp[g].k0) * (L::W.bytes / 1024);
+      for (int kt = 0; kt < kStages && kt < p.grp[g].num_k; ++kt)
+        tma_prefetch_l2(&ms.m[g].w, 0, w_row0 + kt * (L::W.bytes / 1024));
+    }
   }
   // Launched as a programmatic dependent of the preparation: the prologue above overlaps its
   // tail; its outputs are read only after it has completed and flushed.
@@ -448,16 +519,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t armed = 0, last_parity = 0;  // bit s: stage s armed / its last phase parity
       bool ok = true;
-      const uint32_t full_own0 = map_to_rank(full_bar(0), rank);
+      const uint32_t full_own0 = PAIR ? map_to_rank(full_bar(0), rank) : full_bar(0);
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
         const int g = group_of<MAXG>(p, tile), lt = tile - p.grp[g].tile_begin, num_m = p.grp[g].num_m;
         const TmaMaps &maps = ms.m[g];
-        const int m0 = (lt % num_m) * (2 * BM) + (int)rank * BM;  // this CTA's activation rows
-        const int n0 = (lt / num_m) * BN;                          // the pair's output columns
+        const int m0 = PAIR ? (lt % num_m) * (2 * BM) + (int)rank * BM : (lt % num_m) * BM;  // this CTA's rows
+        const int n0 = (lt / num_m) * BN;  // the tile's output columns
         // chunk rows of 1024 bytes; the group's K steps start at k0
         const int a_row0 = ((m0 / 128) * ks_total + p.grp[g].k0) * (L::A.bytes / 1024);
         const int w_row0 = ((n0 / 128 + (int)rank) * ks_total + p.grp[g].k0) * (L::W.bytes / 1024);
         const int num_k = p.grp[g].num_k;
+        // single CTA: the weight chunks of both 128-row halves, by plain bulk copies
+        const uint8_t *w_half0 = p.grp[g].w_tiles + ((size_t)(n0 / 128) * ks_total + p.grp[g].k0) * L::W.bytes;
+        const uint8_t *w_half1 = w_half0 + (size_t)ks_total * L::W.bytes;
         for (int kt = 0; kt < num_k; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, limit, abort_flag)) { ok = false; break; }
           const uint32_t st = smem0 + stage * kStageBytes;
@@ -467,8 +541,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           armed |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           const uint32_t fb = full_own0 + 8u * stage;
-          tma_load_2d(st, &maps.act, 0, a_row0 + kt * (L::A.bytes / 1024), fb);
-          tma_load_2d(st + L::kW, &maps.w, 0, w_row0 + kt * (L::W.bytes / 1024), fb);
+          if (PAIR) {
+            tma_load_2d(st, &maps.act, 0, a_row0 + kt * (L::A.bytes / 1024), fb);
+            tma_load_2d(st + L::kW, &maps.w, 0, w_row0 + kt * (L::W.bytes / 1024), fb);
+          } else {
+            tma_load_2d_1cta(st, &maps.act, 0, a_row0 + kt * (L::A.bytes / 1024), fb);
+            const size_t wk = (size_t)kt * L::W.bytes;
+            bulk_load(st + L::kW, w_half0 + wk, kWCodeBytes, fb);
+            bulk_load(st + L::kW + kWCodeBytes, w_half1 + wk, kWCodeBytes, fb);
+            bulk_load(st + kWScales + kWCodeBytes, w_half0 + wk + kWCodeBytes, L::W.bytes - kWCodeBytes, fb);
+          }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
@@ -513,10 +595,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               // NVFP4: 4 scales per row per MMA (one atom, id 0); MXFP4: 2 (half an atom)
               const uint32_t atom = MX ? (uint32_t)(j >> 1) : (uint32_t)j;
               const uint32_t id = MX ? (uint32_t)(2 * (j & 1)) : 0u;
-              mma_sparse<MX>(acc, dsc(kDescSw64, st4 + (kA + L::A.sp + 32 * j) / 16),
-                             dsc(kDescSw128, st4 + (kW + L::W.b + 64 * j) / 16), t_meta + 2 * j,
-                             idesc_bs(true, MX, id, id), (t_sfa_sp + 4 * atom) | (id << 30),
-                             (t_sfb_sp + 8 * atom) | (id << 30), accumulate);
+              mma_sparse<MX, PAIR>(acc, dsc(kDescSw64, st4 + (kA + L::A.sp + 32 * j) / 16),
+                                   dsc(kDescSw128, st4 + (kW + L::W.b + 64 * j) / 16), t_meta + 2 * j,
+                                   idesc_bs(true, MX, id, id, PAIR), (t_sfa_sp + 4 * atom) | (id << 30),
+                                   (t_sfb_sp + 8 * atom) | (id << 30), accumulate);
               accumulate = 1u;
             }
           }
@@ -524,22 +606,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 4; ++j) {  // four dense MMAs of K = 64 (32 bytes of A and B)
             const uint32_t atom = MX ? (uint32_t)(j >> 1) : (uint32_t)j;
             const uint32_t id = MX ? (uint32_t)(2 * (j & 1)) : 0u;
-            mma_dense<MX>(acc, dsc(kDescSw128, st4 + (kA + L::A.res + 32 * j) / 16),
-                          dsc(kDescSw128, st4 + (kW + L::W.b + 32 * j) / 16), idesc_bs(false, MX, id, id),
-                          (t_sfa_res + 4 * atom) | (id << 30), (t_sfb_res + 8 * atom) | (id << 30), accumulate);
+            mma_dense<MX, PAIR>(acc, dsc(kDescSw128, st4 + (kA + L::A.res + 32 * j) / 16),
+                                dsc(kDescSw128, st4 + (kW + L::W.b + 32 * j) / 16), idesc_bs(false, MX, id, id, PAIR),
+                                (t_sfa_res + 4 * atom) | (id << 30), (t_sfb_res + 8 * atom) | (id << 30), accumulate);
             accumulate = 1u;
           }
-          tc_commit_both(empty_bar(stage));  // frees the stage in both CTAs once these MMAs have read it
-          tc_commit_both(sf_free_bar(buf));  // and the scale buffer in both CTAs
+          tc_commit<PAIR>(empty_bar(stage));  // frees the stage in both CTAs once these MMAs have read it
+          tc_commit<PAIR>(sf_free_bar(buf));  // and the scale buffer in both CTAs
           if (++buf == kScaleBufs) buf = 0;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tc_commit_both(acc_full);
+        tc_commit<PAIR>(acc_full);
         acc_phase ^= 1u;
       }
       // Drain: all MMAs issued above complete before TMEM is released.
-      tc_commit_both(drain_bar);
+      tc_commit<PAIR>(drain_bar);
       volatile uint32_t no_abort = 0;
       mbar_wait(drain_bar, 0, kDrainLimitNs, &no_abort);
     }
@@ -548,14 +630,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;          // TMEM lane quarter this warp may access
     const int col_half = (warp - 2) >> 2;  // columns [128*col_half, 128*col_half + 128)
     const int r_local = quarter * 32 + lane;
-    const uint32_t acc_empty_leader = map_to_rank(acc_empty, 0);
+    const uint32_t acc_empty_leader = PAIR ? map_to_rank(acc_empty, 0) : acc_empty;
     const uint32_t out_smem = smem0 + kOutOffset + (warp - 2) * kStageOutBytes;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs) {
       const int g = group_of<MAXG>(p, tile), lt = tile - p.grp[g].tile_begin, num_m = p.grp[g].num_m;
       const GemmGroup &G = p.grp[g];
       const float s_w = G.tensor_scale[0];
-      const int m0 = (lt % num_m) * (2 * BM) + (int)rank * BM, n0 = (lt / num_m) * BN;
+      const int m0 = PAIR ? (lt % num_m) * (2 * BM) + (int)rank * BM : (lt % num_m) * BM, n0 = (lt / num_m) * BN;
       const int row = m0 + r_local;
       const float scale = row < G.T ? __fmul_rn(G.row_scale[row], s_w) : 0.f;
       if (!mbar_wait_warp(acc_full, acc_phase, limit, abort_flag)) break;
@@ -664,7 +746,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // three tensor-memory buffers with tcgen05.st (registers -> tensor memory), so these writes
     // stay out of the tensor pipe that runs the MMAs in order.
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
-    const uint32_t sf_full_leader0 = map_to_rank(sf_full_bar(0), 0);
+    const uint32_t sf_full_leader0 = PAIR ? map_to_rank(sf_full_bar(0), 0) : sf_full_bar(0);
     int stage = 0;
     uint32_t phase = 0, buf = 0, buf_phase = 0;
     bool ok = true;
@@ -679,13 +761,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t sbuf = tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols + buf * kScaleBufCols;
         const uint32_t t_meta = sbuf, t_sfa_sp = sbuf + 4, t_sfa_res = sbuf + 12, t_sfb_sp = sbuf + 28,
                        t_sfb_res = sbuf + 44;
-        constexpr int kA = 0, kW = L::kW;
+        constexpr int kA = 0;
         // weight scales: the chunk holds the atoms of both 128-row halves of the pair's 256
         // columns (half 0, then half 1); in tensor memory they alternate per atom
-        st_atoms<2 * apt_res>(t_sfb_res, st + kW + L::W.sf_res,
+        st_atoms<2 * apt_res>(t_sfb_res, st + kWScales + L::W.sf_res,
                               [&](int i) { return ((i & 1) * apt_res + (i >> 1)) * 512; }, lane);
         if (SPARSE)
-          st_atoms<2 * apt_sp>(t_sfb_sp, st + kW + L::W.sf_sp,
+          st_atoms<2 * apt_sp>(t_sfb_sp, st + kWScales + L::W.sf_sp,
                                [&](int i) { return ((i & 1) * apt_sp + (i >> 1)) * 512; }, lane);
         st_atoms<apt_res>(t_sfa_res, st + kA + L::A.sf_res, [&](int i) { return i * 512; }, lane);
         if (SPARSE) {
@@ -714,9 +796,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // cluster barrier.
   __syncwarp();
   tc_fence_before();
-  cluster_sync();
+  block_sync<PAIR>();
   tc_fence_after();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  if (warp == 1) tmem_dealloc<PAIR>(tmem);
+}
+
+template <bool MX, bool SPARSE, int MAXG>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    sharq_gemm_kernel(const __grid_constant__ TmaMapSet<MAXG> ms, const __grid_constant__ GemmParams p) {
+  gemm_body<MX, SPARSE, MAXG, true>(ms, p);
+}
+
+// One CTA per 128 x 256 tile (no cluster).
+template <bool MX, bool SPARSE, int MAXG>
+__global__ void __launch_bounds__(kThreads, 1)
+    sharq_gemm1_kernel(const __grid_constant__ TmaMapSet<MAXG> ms, const __grid_constant__ GemmParams p) {
+  gemm_body<MX, SPARSE, MAXG, false>(ms, p);
 }
 
 // ---------------------------------------------------------------- tensor-core peak loop
@@ -932,7 +1027,7 @@ struct MapCache {
 
 constexpr int kMaxDevices = 64;
 
-template <bool MX, bool SPARSE, int MAXG>
+template <bool MX, bool SPARSE, int MAXG, bool PAIR>
 cudaError_t launch_t(const TmaMapSet<MAXG> &ms, const GemmParams &p, cudaStream_t st) {
   static std::once_flag once[kMaxDevices];
   static cudaError_t setup_err[kMaxDevices];
@@ -941,26 +1036,29 @@ cudaError_t launch_t(const TmaMapSet<MAXG> &ms, const GemmParams &p, cudaStream_
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::call_once(once[dev], [dev] {
-    setup_err[dev] = cudaFuncSetAttribute(sharq_gemm_kernel<MX, SPARSE, MAXG>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  auto kern = PAIR ? sharq_gemm_kernel<MX, SPARSE, MAXG> : sharq_gemm1_kernel<MX, SPARSE, MAXG>;
+  constexpr int smem = PAIR ? kSmemBytes : kSmemBytes1;
+  std::call_once(once[dev], [dev, kern] {
+    setup_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (setup_err[dev] == cudaSuccess)
       setup_err[dev] = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
   });
   if (setup_err[dev] != cudaSuccess) return setup_err[dev];
   if (p.num_tiles == 0) return cudaSuccess;
-  const int pairs = p.num_tiles < sms[dev] / 2 ? p.num_tiles : sms[dev] / 2;
+  // persistent: one CTA pair per two SMs, or one CTA per SM, at most one per tile
+  const int units = PAIR ? sms[dev] / 2 : sms[dev];
+  const int grid = (p.num_tiles < units ? p.num_tiles : units) * (PAIR ? 2 : 1);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs);
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may start while the previous kernel drains
   attr.val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, sharq_gemm_kernel<MX, SPARSE, MAXG>, ms, p);
+  e = cudaLaunchKernelEx(&cfg, kern, ms, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1003,19 +1101,44 @@ cudaError_t launch_groups(const GemmParams &p, cudaStream_t st, const char **why
       return cudaErrorInvalidValue;
     }
   const bool mx = p.fmt == kFmtMX;
-  if (p.sparse) return mx ? launch_t<true, true, MAXG>(ms, p, st) : launch_t<false, true, MAXG>(ms, p, st);
-  return mx ? launch_t<true, false, MAXG>(ms, p, st) : launch_t<false, false, MAXG>(ms, p, st);
+  if (p.sparse && p.single)
+    return mx ? launch_t<true, true, MAXG, false>(ms, p, st) : launch_t<false, true, MAXG, false>(ms, p, st);
+  if (p.sparse) return mx ? launch_t<true, true, MAXG, true>(ms, p, st) : launch_t<false, true, MAXG, true>(ms, p, st);
+  return mx ? launch_t<true, false, MAXG, true>(ms, p, st) : launch_t<false, false, MAXG, true>(ms, p, st);
 }
 
 }  // namespace
+
+// Single-CTA tiles (128 rows) against CTA-pair tiles (256 rows) for a sparse launch: the one
+// whose rounds of tiles over the persistent grid take less time, a single-CTA tile costing
+// 1.1 pair tiles (it moves both weight halves into one SM: measured ~7 % slower at equal
+// rounds). A problem of at most 128 rows pads a pair tile by half; the single-CTA form wins
+// where that padding adds rounds (a mixture-of-experts layer, a split-K launch), not for a
+// lone small launch that fits in one round either way.
+bool use_single_cta(const GemmParams &p) {
+  if (!p.sparse) return false;
+  const int sms = sm_count();
+  if (sms < 2) return false;
+  const long long num_n = (p.N + BN - 1) / BN;
+  long long pair_tiles = 0, single_tiles = 0;
+  for (int g = 0; g < p.n_groups; ++g) {
+    pair_tiles += (p.grp[g].T + 2 * BM - 1) / (2 * BM) * num_n;
+    single_tiles += (p.grp[g].T + BM - 1) / BM * num_n;
+  }
+  const long long pair_rounds = (pair_tiles + sms / 2 - 1) / (sms / 2);
+  const long long single_rounds = (single_tiles + sms - 1) / sms;
+  return 10 * pair_rounds > 11 * single_rounds;
+}
 
 // Fills the tile ranges of p.grp[0 .. n_groups) and launches one kernel.
 cudaError_t launch_gemm(GemmParams p, cudaStream_t st, const char **why) {
   int tiles = 0;
   const int num_n = (p.N + BN - 1) / BN;
+  p.single = use_single_cta(p) ? 1 : 0;
+  const int rows_per_tile = p.single ? BM : 2 * BM;
   for (int g = 0; g < p.n_groups; ++g) {
     if (p.grp[g].num_k == 0) p.grp[g].num_k = p.K / BK - p.grp[g].k0;
-    p.grp[g].num_m = (p.grp[g].T + 2 * BM - 1) / (2 * BM);
+    p.grp[g].num_m = (p.grp[g].T + rows_per_tile - 1) / rows_per_tile;
     p.grp[g].tile_begin = tiles;
     tiles += p.grp[g].num_m * num_n;
   }
@@ -1038,15 +1161,19 @@ int sm_count() {
   return sms[dev];
 }
 
-// Slices for a (tokens x n_out x k) linear, from a cost estimate: a pair spends about 0.5 us
-// per K step of a tile (the tensor pipe's rate at these tile sizes), so one slice of q steps
-// saves (K steps - q) * 0.5 us when every pair holds at most one tile; the split form costs a
+// Slices for a (tokens x n_out x k) linear, from a cost estimate: a pair (or, for at most 128
+// rows, a single CTA) spends about 0.5 us per K step of a tile (the tensor pipe's rate at these
+// tile sizes), so one slice of q steps saves (K steps - q) * 0.5 us when every unit holds at
+// most one tile; the split form costs a
 // second launch (~3 us) and the float32 partials written and read back (S * tokens * n_out *
 // 8 bytes at ~3 TB/s, L2-resident). 1 when the tiles already fill half of the SM pairs or
 // slicing does not pay; at most kMaxGroups slices, at least 2 K steps each.
 int gemm_split_count(int tokens, int n_out, int k) {
-  const int pairs = sm_count() / 2;
-  const int tiles = ((tokens + 2 * BM - 1) / (2 * BM)) * ((n_out + BN - 1) / BN);
+  // at most 128 rows: the single-CTA form (one 128-row tile per SM), else CTA pairs
+  const bool single = tokens <= BM;
+  const int pairs = single ? sm_count() : sm_count() / 2;
+  const int rows = single ? BM : 2 * BM;
+  const int tiles = ((tokens + rows - 1) / rows) * ((n_out + BN - 1) / BN);
   const int ks = k / BK;
   if (pairs < 2 || 2 * tiles > pairs) return 1;
   int s_max = pairs / tiles;

@@ -91,6 +91,7 @@ struct GemmParams {
   int n_groups, num_tiles;    // num_tiles: pair tiles over all groups
   int N, K, N_pad;            // shared by every group
   int fmt, out_f32, sparse;
+  int single;                 // one CTA per 128 x 256 tile (set by launch_gemm), else CTA pairs
   long long wait_limit;
 };
 

@@ -55,7 +55,7 @@ def test_split_not_called_for_and_small_workspace():
     S = require_gpu()
     assert S.sharq_linear_workspace_size(2048, 6144, 4096) == 0  # enough tiles already
     assert S.sharq_linear_workspace_size(1, 16, 256) == 0        # one K step
-    assert S.sharq_linear_workspace_size(128, 3584, 3584) == 0   # partials would cost more than slicing saves
+    assert S.sharq_linear_workspace_size(256, 3584, 3584) == 0   # partials would cost more than slicing saves
     p, wp, cols, ref = _problem(S, 300, 512, 768, 0, 9)
     ws = torch.full((64,), 0x33, dtype=torch.uint8, device="cuda")
     y = S.sharq_linear(p, wp, out_dtype=torch.float32, workspace=ws)  # plain launch
