@@ -435,14 +435,16 @@ def run_sharq(args, rank, world, local):
     sw_bytes = T * Kd * (4 + PREP_BYTES_PER_ELEM - 2) + T * 4
     # ---- mixture of experts: Qwen3-30B-A3B expert gate/up projections (K=2048, N=2*768) for
     # T tokens routed top-8 of 128. The routed rows are laid out expert by expert, each
-    # expert's group padded to 256 rows, prepared by ONE sharq_prepare over all of them, and
-    # every expert's view of that buffer goes to one grouped GEMM launch.
+    # expert's group padded to 128 rows (a chunk row block), prepared by ONE sharq_prepare over
+    # all of them, and every expert's view of that buffer goes to one grouped GEMM launch. A
+    # view reads up to 256 rows of chunks from its start (a pair tile), so the buffer keeps 256
+    # rows of slack at its end.
     moe = wl.QWEN3_MOE
     Km, Nm, E = moe["hidden"], 2 * moe["moe_intermediate"], moe["n_experts"]
     route = wl.moe_routing(replica_seed(rank), T, E, moe["top_k"])
     counts = np.bincount(route.reshape(-1), minlength=E)
-    starts = np.concatenate([[0], np.cumsum((counts + 255) // 256 * 256)])[:-1]
-    rows_pad = int(starts[-1] + (counts[-1] + 255) // 256 * 256)
+    starts = np.concatenate([[0], np.cumsum((counts + 127) // 128 * 128)])[:-1]
+    rows_pad = int(starts[-1] + (counts[-1] + 127) // 128 * 128)
     order = np.argsort(route.reshape(-1), kind="stable")            # assignments sorted by expert
     src_tok = (order // moe["top_k"]).astype(np.int64)
     dst_row = np.concatenate([starts[e] + np.arange(counts[e]) for e in range(E)]).astype(np.int64)
@@ -456,8 +458,9 @@ def run_sharq(args, rank, world, local):
         w_e = (torch.randn(Nm, Km, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)
         wps_moe.append(S.sharq_pack_weight(w_e, "nvfp4"))
     del w_e
-    p_moe = S.alloc_prep(rows_pad, Km, 2, 4, 2, "nvfp4")
-    chunk = p_moe.tiles.numel() // (rows_pad // 128)               # bytes per 128-row block
+    p_moe = S.alloc_prep(rows_pad + 256, Km, 2, 4, 2, "nvfp4")    # + slack for the last view
+    p_moe.tokens, p_moe.row_scale = rows_pad, p_moe.row_scale[:rows_pad]
+    chunk = S.sharq_prep_buffer_sizes(256, Km, 2, 4, 2, "nvfp4")[0] // 2  # bytes per 128-row block
     views = [S.Prep(p_moe.tiles[int(starts[e]) // 128 * chunk:], p_moe.row_scale[int(starts[e]):],
                     int(counts[e]), Km, 2, 4, 2, S.SHARQ_NVFP4) for e in range(E)]
     ys_moe = [torch.empty(max(int(c), 1), Nm, dtype=torch.bfloat16, device="cuda") for c in counts]

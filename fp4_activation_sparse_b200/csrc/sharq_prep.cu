@@ -1,10 +1,9 @@
 // Fused SharQ preparation operator (K2) and the dense FP4 activation quantizer.
 //
-// "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM Inference",
-// Abstract: "a fused preparation kernel absorbs mask generation, residual
-// construction, and layer normalization into one operator"; the residual is
-// defined "relative to the quantized sparse backbone rather than the
-// unquantized sparse values".
+// Per "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM Inference"
+// (Abstract), one kernel performs the normalization, the choice of the mask and the
+// construction of the residual; the residual is taken against the backbone after its FP4
+// rounding, not against the backbone's unrounded values.
 //
 // One read of the bf16 activations. A team of W warps owns one token row (W = K/4096
 // rounded up); every lane owns "double pieces" of 16 consecutive K elements (one 256-bit

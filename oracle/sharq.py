@@ -9,8 +9,8 @@ Quantization for LLM Inference", Abstract): for each activation tensor,
 
 1. optional layer normalization (RMSNorm; the README's "--disable_rmsnorm_fusion"
    flag, section "Evaluation"),
-2. an input-adaptive N:M mask that extracts an outlier-dominated sparse
-   backbone,
+2. an N:M mask chosen from the activation itself, which pulls the outliers
+   into a sparse backbone,
 3. FP4 quantization of that backbone,
 4. a dense residual defined against the *quantized* backbone (not the
    unquantized sparse values), quantized densely to FP4,
@@ -264,8 +264,8 @@ def prepare(x, gamma, eps: float, n: int, m: int, unit: int, fmt: str, per_tenso
 # --------------------------------------------------------------------------------------
 # SwiGLU fused into the preparation operator (down-projection input)
 # --------------------------------------------------------------------------------------
-# The abstract's fused preparation kernel absorbs the steps in front of the quantizer into
-# one operator; for a down projection that step is the gated activation x = SiLU(g) * u of
+# The abstract folds the steps in front of the quantizer into the one preparation kernel;
+# for a down projection that step is the gated activation x = SiLU(g) * u of
 # the gate/up projection's output [g | u]. Reading (the pages give no formula): the
 # activation the unfused pipeline hands to the down projection is bf16, so
 #   x = bf16_RNE(fp32(silu(g) * u)),  silu(g) = fp32(g * sigma(g)),

@@ -8,9 +8,9 @@ Wan2.2-T2V-A14B ("SharQ: Bridging Activation Sparsity and FP4 Quantization for
 LLM Inference", Abstract) with wikitext2 / lm-eval suites (README, section
 "Evaluation"). None of those weights or datasets exist here; these generators
 stand in for them with the models' layer shapes and with activations that have
-the property the abstract names: "input-dependent outliers that dominate
-block scales" -- a few outlier channels scaled by large factors, times a
-log-normal per-token scale.
+the property the abstract attributes to real ones: outliers, varying from input to
+input, large enough to set the block scales -- here a few outlier channels scaled by
+large factors, times a log-normal per-token scale.
 
 Values are drawn in float32 with numpy's PCG64 (``default_rng(seed)``) and
 rounded to bf16 (round to nearest even) by integer bit operations, so the
