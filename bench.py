@@ -482,9 +482,25 @@ def run_sharq(args, rank, world, local):
     p_ts = S.alloc_prep(T, K, 2, 4, 2, "nvfp4")
     ws_ts = torch.zeros(S.sharq_tensor_scale_workspace_size(T, K), dtype=torch.uint8, device="cuda")
     torch.cuda.synchronize()
-    t_ts = graph_time(capture(lambda st: [S.sharq_prepare_tensor_scale(xs[s], gamma, lin.eps, out=p_ts,
-                                                                       workspace=ws_ts, stream=st)
-                                          for s in range(nsets)]), nsets)
+    g_ts = capture(lambda st: [S.sharq_prepare_tensor_scale(xs[s], gamma, lin.eps, out=p_ts, workspace=ws_ts,
+                                                            stream=st) for s in range(nsets)])
+    # the per-row preparation timed again beside it (same clock and cache state), alternating
+    t_ts, t_row_here = [], []
+    for _ in range(3):
+        t_ts.append(graph_time(g_ts, nsets))
+        t_row_here.append(graph_time(prep_graph, nsets))
+    t_ts, t_row_here = min(t_ts), min(t_row_here)
+    # ... and at 16384 rows, where the rows no longer fit on chip and phase 2 re-reads x
+    x16 = wl.outlier_activations_device(replica_seed(rank) + 700, 16384, K, 41, 20.0, 100.0, 0.5)
+    p16, pts16 = S.alloc_prep(16384, K, 2, 4, 2, "nvfp4"), S.alloc_prep(16384, K, 2, 4, 2, "nvfp4")
+    ws16 = torch.zeros(S.sharq_tensor_scale_workspace_size(16384, K), dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    g_row16 = capture(lambda st: S.sharq_prepare(x16, gamma, lin.eps, out=p16, stream=st))
+    g_ts16 = capture(lambda st: S.sharq_prepare_tensor_scale(x16, gamma, lin.eps, out=pts16, workspace=ws16,
+                                                             stream=st))
+    t_row16 = min(graph_time(g_row16, 1) for _ in range(2))
+    t_ts16 = min(graph_time(g_ts16, 1) for _ in range(2))
+    del x16, p16, pts16, ws16
     sw_gbs = sw_bytes / (t_sw / 1e3) / 1e9
     del gus
 
@@ -672,8 +688,10 @@ def run_sharq(args, rank, world, local):
             "frac": sw_gbs / hbm_peak, "unfused_torch_swiglu_plus_prep_us": t_unf * 1e3},
             "tensor_scale_prep": {
                 "workload": f"llama31_8b_qkv_prefill T={T} K={K} nvfp4 2:4-pairs fused-rmsnorm, one scale per tensor",
-                "t_us": t_ts * 1e3, "per_row_scale_prep_us": t_prep_ms * 1e3,
-                "ratio_to_per_row": t_ts / t_prep_ms,
+                "t_us": t_ts * 1e3, "per_row_scale_prep_us": t_row_here * 1e3,
+                "ratio_to_per_row": t_ts / t_row_here,
+                "t_us_16384_rows": t_ts16 * 1e3, "per_row_scale_prep_us_16384_rows": t_row16 * 1e3,
+                "ratio_to_per_row_16384_rows": t_ts16 / t_row16,
                 "note": "one cooperative launch (phase 1 rstd + amax, grid barrier, phase 2 quantize; every row "
                         "stays in registers at this size, x read once); the workspace's barrier words reset themselves"},
             "moe_grouped": moe_line,

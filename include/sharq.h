@@ -244,13 +244,19 @@ int sharq_linear_split(const sharq_prep *a, const sharq_wpack *w, void *y_dev, i
                        void *workspace_dev, size_t workspace_bytes, void *stream);
 
 /* Grouped (mixture-of-experts) SharQ linear: n_groups independent problems
- * Y_e = sharq_linear(a[e], w[e]) computed by one launch per 64 groups, the CTA pairs working
- * through the output tiles of all groups (each expert's tokens prepared by sharq_prepare into
- * their own buffers, so no tile mixes experts). The abstract evaluates a mixture-of-experts
- * model (Qwen3-30B-A3B) with the method; this is its expert layer.
+ * Y_e = sharq_linear(a[e], w[e]) computed by one launch per 64 groups, the persistent grid
+ * working through the output tiles of all groups (no tile mixes experts). When the groups are
+ * mostly at most 128 rows the launch runs on single-CTA 128-row tiles instead of CTA-pair
+ * 256-row tiles (chosen per launch, same results up to float32 rounding order). The abstract
+ * evaluates a mixture-of-experts model (Qwen3-30B-A3B) with the method; this is its expert
+ * layer.
  *   a[e], w[e]  prepared activation and packed weight of group e; every weight has the same
  *               n_out, k and fmt; a[e].tokens == 0 marks an expert without tokens (skipped:
- *               its prep buffers and y_dev[e] are not used and may be NULL)
+ *               its prep buffers and y_dev[e] are not used and may be NULL). a[e].tiles may
+ *               point into a larger prepared buffer at any 128-row block (one sharq_prepare
+ *               over all experts' rows laid out expert by expert): the GEMM reads up to
+ *               round_up(tokens, 256) rows of chunks from there (rows past the expert's own are
+ *               read, never written), so that many rows must lie inside the allocation.
  *   y_dev[e]    [a[e].tokens][n_out] output of group e (bf16 or float32 per out_dtype)
  * Checks and errors as sharq_linear, per group. */
 int sharq_linear_grouped(const sharq_prep *a, const sharq_wpack *w, void *const *y_dev, int n_groups,
