@@ -99,3 +99,20 @@ def test_tensor_scale_several_row_groups_per_block(T, K, norm):
         assert abs(int(got["row_scale"][0].view(np.int32)) - int(ref["row_scale"][0].view(np.int32))) <= 1
         for key in ("sp_codes", "res_codes", "idx"):
             assert np.mean(got[key] != ref[key]) <= 1e-4, key
+
+
+def test_tensor_scale_benchmark_launch():
+    """The benchmark's per-tensor launch (Llama-3.1-8B QKV input, 2048 x 4096, fused RMSNorm):
+    the whole tensor against the oracle (the one-ulp rstd allowance of the per-row operator)."""
+    S = require_gpu()
+    lin = wl.llama_qkv(T=2048)
+    ws = torch.zeros(S.sharq_tensor_scale_workspace_size(2048, 4096), dtype=torch.uint8, device="cuda")
+    p = S.sharq_prepare_tensor_scale(to_dev_bf16(lin.x), to_dev_bf16(lin.gamma), lin.eps, workspace=ws)
+    torch.cuda.synchronize()
+    assert S.sharq_device_status() == S.SHARQ_OK
+    got = hw.read_prep(p, 16)
+    ref = O.prepare(f32(lin.x), f32(lin.gamma), lin.eps, 2, 4, 2, O.NVFP4, per_tensor=True)
+    assert np.all(got["row_scale"] == got["row_scale"][0])
+    assert abs(int(got["row_scale"][0].view(np.int32)) - int(ref["row_scale"][0].view(np.int32))) <= 1
+    for key in ("sp_codes", "res_codes", "idx", "sp_scales", "res_scales"):
+        assert np.mean(got[key] != ref[key]) <= 1e-4, key
