@@ -489,7 +489,9 @@ __device__ __forceinline__ void row_scales(int fmt, float amax, float &s_x, floa
 constexpr int kRow = 0, kSwiglu = 1;
 
 template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE, int DP>
-__global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
+// Two blocks per SM: the register cap keeps the branch-free piece loop below from costing
+// occupancy (a few bytes of spill at 8 pieces per lane with RMSNorm).
+__global__ void __launch_bounds__(256, 2) prep_kernel(PrepParams p) {
   extern __shared__ float4 gamma_smem4[];  // NORM: the RMSNorm weight as float32 (K rounded up to 512)
   __shared__ double sm_d[64];
   __shared__ float sm_f[64];
@@ -568,6 +570,19 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   uint8_t *chunk0 = p.tiles + ((size_t)(row >> 7) * p.KS + 2 * wt + (lane >> 4)) * kChunk;
   const size_t chunk_step = (size_t)2 * W * kChunk;
   const bool pad_row = !live_row && row < p.T_pad;
+  if (live_row && ndp_row == DP * stride) {
+    // Every piece of the row is live (K a multiple of 512 W): no per-piece control flow, so
+    // the compiler may interleave pieces (10 % faster at 2048 rows, 8 % at 16384).
+#pragma unroll
+    for (int i = 0; i < DP; ++i) {
+      float v[16];
+      unpack16(xr[i], v);
+      if (NORM) normalize16<false>(v, g_lane + i * 128 * W, rstd);
+      process16<FMT, UNIT, DENSE>(chunk0 + i * chunk_step, o, v, true, s_x, g_x);
+    }
+    if (wt == 0 && lane == 0) p.row_scale[row] = s_x;
+    return;
+  }
 #pragma unroll
   for (int i = 0; i < DP; ++i) {
     const int base = i * stride + wt * 32;  // warp-uniform
@@ -754,6 +769,16 @@ __global__ void __launch_bounds__(256, 2) prep_tensor_kernel(PrepParams p, uint3
     uint8_t *chunk0 = p.tiles + ((size_t)(row >> 7) * p.KS + 2 * wt + (lane >> 4)) * kChunk;
     const size_t chunk_step = (size_t)2 * W * kChunk;
     const bool pad_row = !live_row && row < p.T_pad;
+    if (live_row && ndp_row == DP * stride) {  // every piece live: branch-free (as prep_kernel)
+#pragma unroll
+      for (int i = 0; i < DP; ++i) {
+        float v[16];
+        unpack16(xr[i], v);
+        if (NORM) normalize16<false>(v, g_lane + i * 128 * W, rstd);
+        process16<kFmtNV, UNIT, false>(chunk0 + i * chunk_step, o, v, true, s_x, g_x);
+      }
+      continue;
+    }
 #pragma unroll
     for (int i = 0; i < DP; ++i) {
       const int base = i * stride + wt * 32;  // warp-uniform
