@@ -570,9 +570,11 @@ __global__ void __launch_bounds__(256, 2) prep_kernel(PrepParams p) {
   uint8_t *chunk0 = p.tiles + ((size_t)(row >> 7) * p.KS + 2 * wt + (lane >> 4)) * kChunk;
   const size_t chunk_step = (size_t)2 * W * kChunk;
   const bool pad_row = !live_row && row < p.T_pad;
-  if (live_row && ndp_row == DP * stride) {
+  if (p.unrolled && live_row && ndp_row == DP * stride) {
     // Every piece of the row is live (K a multiple of 512 W): no per-piece control flow, so
-    // the compiler may interleave pieces (10 % faster at 2048 rows, 8 % at 16384).
+    // the compiler may interleave pieces (8 % faster at 16384 rows). The loop's code is
+    // larger, so a launch of one wave, whose blocks all start with a cold instruction cache,
+    // keeps the loop below (the same speed in the benchmark's step at 2048 rows).
 #pragma unroll
     for (int i = 0; i < DP; ++i) {
       float v[16];
@@ -769,7 +771,9 @@ __global__ void __launch_bounds__(256, 2) prep_tensor_kernel(PrepParams p, uint3
     uint8_t *chunk0 = p.tiles + ((size_t)(row >> 7) * p.KS + 2 * wt + (lane >> 4)) * kChunk;
     const size_t chunk_step = (size_t)2 * W * kChunk;
     const bool pad_row = !live_row && row < p.T_pad;
-    if (live_row && ndp_row == DP * stride) {  // every piece live: branch-free (as prep_kernel)
+    // every piece live and several row groups per block (the instruction cache warm after the
+    // first): branch-free, as prep_kernel's multi-wave launches
+    if (J > 1 && live_row && ndp_row == DP * stride) {
 #pragma unroll
       for (int i = 0; i < DP; ++i) {
         float v[16];
@@ -808,12 +812,25 @@ __global__ void __launch_bounds__(256, 2) prep_tensor_kernel(PrepParams p, uint3
   }
 }
 
+int prep_sm_count() {
+  static std::once_flag once[64];
+  static int sms[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::call_once(once[dev], [dev] {
+    if (cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms[dev] = 148;
+  });
+  return sms[dev];
+}
+
 template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE, int DP>
 cudaError_t launch_k(const PrepParams &p, cudaStream_t st) {
   const int W = p.TS;
   const int teams = W >= 8 ? 1 : 8 / W;
   const int block = teams * W * 32;
   const int grid = (p.T_pad + teams - 1) / teams;
+  PrepParams q = p;
+  q.unrolled = grid >= 4 * prep_sm_count() ? 1 : 0;  // several waves: the branch-free loop pays
   // the staging layout reserves 512 floats per 32 double pieces: round K up to 512
   const size_t smem = NORM ? (size_t)((p.K + 511) / 512 * 512) * sizeof(float) : 0;
   if (smem > 48 * 1024) {
@@ -830,7 +847,7 @@ cudaError_t launch_k(const PrepParams &p, cudaStream_t st) {
     });
     if (err[dev] != cudaSuccess) return err[dev];
   }
-  prep_kernel<FMT, UNIT, NORM, DENSE, MODE, DP><<<grid, block, smem, st>>>(p);
+  prep_kernel<FMT, UNIT, NORM, DENSE, MODE, DP><<<grid, block, smem, st>>>(q);
   return cudaGetLastError();
 }
 

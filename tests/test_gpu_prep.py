@@ -193,3 +193,26 @@ def test_prep_full_size_sampled_rows(which, T):
         assert_close_norm(sub, ref, f32(lin.x[rows]), f32(lin.gamma), lin.eps)
     else:
         assert_exact(sub, ref)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("unit", [2, 1])
+@pytest.mark.parametrize("use_norm", [False, True])
+def test_prep_multiwave_full_rows_sampled(fmt, unit, use_norm):
+    """A launch of several waves (6000 rows of K=2048: 750 blocks for 148 SMs) with every piece
+    of a row live takes the branch-free piece loop; sampled rows against the oracle."""
+    S = require_gpu()
+    rng = np.random.default_rng(60 + fmt + 2 * unit)
+    T, K = 6000, 2048
+    x_bits = wl.outlier_activations(rng, T, K, K // 100, 20.0, 100.0, 0.5)
+    g_bits = wl.rms_gamma(rng, K)
+    p = S.sharq_prepare(to_dev_bf16(x_bits), to_dev_bf16(g_bits) if use_norm else None, 1e-6, 2, 4, unit, fmt)
+    torch.cuda.synchronize()
+    got_all = hw.read_prep(p, O.block_size(FMT_NAME[fmt]))
+    rows = np.unique(np.concatenate([[0, 127, 128, T - 1], rng.choice(T, 40, replace=False)]))
+    got = {k: v[rows] for k, v in got_all.items()}
+    ref = O.prepare(f32(x_bits[rows]), f32(g_bits) if use_norm else None, 1e-6, 2, 4, unit, FMT_NAME[fmt])
+    if use_norm:
+        assert_close_norm(got, ref, f32(x_bits[rows]), f32(g_bits), 1e-6)
+    else:
+        assert_exact(got, ref)
