@@ -58,7 +58,6 @@ struct PrepParams {
   int T, K, T_pad;
   int KS;  // 256-K steps per row
   int TS;  // warps per row team
-  int unrolled;  // take the branch-free piece loop for full rows (launches of several waves)
   uint8_t *tiles;         // activation chunks (act_tile layout)
   float *row_scale;       // [T]
 };

@@ -488,9 +488,11 @@ __device__ __forceinline__ void row_scales(int fmt, float amax, float &s_x, floa
 // the input formed as SiLU(g)*u from [g | u].
 constexpr int kRow = 0, kSwiglu = 1;
 
-template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE, int DP>
-// Two blocks per SM: the register cap keeps the branch-free piece loop below from costing
-// occupancy (a few bytes of spill at 8 pieces per lane with RMSNorm).
+// UNROLLED: the branch-free piece loop for rows whose every piece is live, in its own
+// instantiation (the other instantiations hold only the per-piece loop). Two blocks per SM:
+// the register cap keeps 16 warps per SM (the branch-free loop alone would take ~142
+// registers; capped, a few bytes spill).
+template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE, int DP, bool UNROLLED>
 __global__ void __launch_bounds__(256, 2) prep_kernel(PrepParams p) {
   extern __shared__ float4 gamma_smem4[];  // NORM: the RMSNorm weight as float32 (K rounded up to 512)
   __shared__ double sm_d[64];
@@ -570,7 +572,7 @@ __global__ void __launch_bounds__(256, 2) prep_kernel(PrepParams p) {
   uint8_t *chunk0 = p.tiles + ((size_t)(row >> 7) * p.KS + 2 * wt + (lane >> 4)) * kChunk;
   const size_t chunk_step = (size_t)2 * W * kChunk;
   const bool pad_row = !live_row && row < p.T_pad;
-  if (p.unrolled && live_row && ndp_row == DP * stride) {
+  if (UNROLLED && live_row && ndp_row == DP * stride) {
     // Every piece of the row is live (K a multiple of 512 W): no per-piece control flow, so
     // the compiler may interleave pieces (8 % faster at 16384 rows). The loop's code is
     // larger, so a launch of one wave, whose blocks all start with a cold instruction cache,
@@ -823,14 +825,13 @@ int prep_sm_count() {
   return sms[dev];
 }
 
-template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE, int DP>
-cudaError_t launch_k(const PrepParams &p, cudaStream_t st) {
+template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE, int DP, bool UNROLLED>
+cudaError_t launch_u(const PrepParams &p, cudaStream_t st) {
   const int W = p.TS;
   const int teams = W >= 8 ? 1 : 8 / W;
   const int block = teams * W * 32;
   const int grid = (p.T_pad + teams - 1) / teams;
-  PrepParams q = p;
-  q.unrolled = grid >= 4 * prep_sm_count() ? 1 : 0;  // several waves: the branch-free loop pays
+  const PrepParams &q = p;
   // the staging layout reserves 512 floats per 32 double pieces: round K up to 512
   const size_t smem = NORM ? (size_t)((p.K + 511) / 512 * 512) * sizeof(float) : 0;
   if (smem > 48 * 1024) {
@@ -842,13 +843,30 @@ cudaError_t launch_k(const PrepParams &p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [dev] {
-      err[dev] = cudaFuncSetAttribute(prep_kernel<FMT, UNIT, NORM, DENSE, MODE, DP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      err[dev] = cudaFuncSetAttribute(prep_kernel<FMT, UNIT, NORM, DENSE, MODE, DP, UNROLLED>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       32768 * (int)sizeof(float));
     });
     if (err[dev] != cudaSuccess) return err[dev];
   }
-  prep_kernel<FMT, UNIT, NORM, DENSE, MODE, DP><<<grid, block, smem, st>>>(q);
+  prep_kernel<FMT, UNIT, NORM, DENSE, MODE, DP, UNROLLED><<<grid, block, smem, st>>>(q);
   return cudaGetLastError();
+}
+
+// The branch-free instantiation for the executed mask (pairs, sparse) when every piece of a
+// row is live and the launch has several waves (grid >= 4 x the SM count: the instruction
+// cache is warm after the first blocks; a one-wave launch starts every block cold and the
+// larger loop then costs as much as it saves).
+template <int FMT, int UNIT, bool NORM, bool DENSE, int MODE, int DP>
+cudaError_t launch_k(const PrepParams &p, cudaStream_t st) {
+  const int W = p.TS;
+  const int teams = W >= 8 ? 1 : 8 / W;
+  const int grid = (p.T_pad + teams - 1) / teams;
+  const bool full = (p.K >> 4) == DP * 32 * W;
+  if constexpr (UNIT == 2 && !DENSE) {
+    if (full && grid >= 4 * prep_sm_count()) return launch_u<FMT, UNIT, NORM, DENSE, MODE, DP, true>(p, st);
+  }
+  return launch_u<FMT, UNIT, NORM, DENSE, MODE, DP, false>(p, st);
 }
 
 // A single-warp row of at most 2048 elements needs 4 pieces per lane: the smaller register
