@@ -81,13 +81,14 @@ def test_dit_linear():
     print(check_shape(S, lin.x, lin.w, 0))
 
 
-@pytest.mark.parametrize("counts", [[130, 0, 256, 77, 300], [5, 128, 0, 77, 64, 100, 1, 128]])
-def test_moe_grouped_at_expert_shape(counts):
+@pytest.mark.parametrize("counts,fmt", [([130, 0, 256, 77, 300], 0), ([5, 128, 0, 77, 64, 100, 1, 128], 0),
+                                        ([5, 128, 0, 77, 64, 100, 1, 128] * 3, 1)])
+def test_moe_grouped_at_expert_shape(counts, fmt):
     """Qwen3-30B-A3B experts (K=2048, N=2*768): ragged and empty experts in one grouped launch;
     the second set (every expert at most 128 rows) runs on single-CTA 128-row tiles."""
     S = require_gpu()
     K, N = wl.QWEN3_MOE["hidden"], 2 * wl.QWEN3_MOE["moe_intermediate"]
-    preps, wps, refs = _experts(S, np.random.default_rng(77), counts, K, N, 0)
+    preps, wps, refs = _experts(S, np.random.default_rng(77), counts, K, N, fmt)
     ys = [torch.empty(max(t, 1), N, dtype=torch.float32, device="cuda") for t in counts]
     S.sharq_linear_grouped(preps, wps, ys)
     torch.cuda.synchronize()
