@@ -14,8 +14,10 @@
  *
  * Conventions for every call:
  *  - Pointers named *_dev are device pointers; the caller allocates and owns all
- *    of them (sizes from sharq_prep_buffer_sizes / sharq_wpack_buffer_sizes).
- *    The library allocates no memory and never synchronizes the stream.
+ *    of them (sizes from sharq_prep_buffer_sizes / sharq_wpack_buffer_sizes and the
+ *    workspace-size queries). The library allocates no memory and never synchronizes the
+ *    stream; its only device memory of its own is the 8 KB static array that
+ *    sharq_prepare_tensor_scale_noalloc uses in place of a workspace.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Work is enqueued asynchronously on it.
  *  - Every argument is checked on the host before any launch. A call returns
