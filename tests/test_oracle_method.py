@@ -158,7 +158,8 @@ def test_zero_block_gives_zero_codes_and_scale():
 
 
 # ------------------------------------------------------------------ preparation: golden rows
-@pytest.mark.parametrize("name", ["nvfp4_pair24_row.txt", "nvfp4_elem24_row.txt", "mxfp4_pair24_row.txt"])
+@pytest.mark.parametrize("name", ["nvfp4_pair24_row.txt", "nvfp4_elem24_row.txt", "mxfp4_pair24_row.txt",
+                                  "mxfp4_elem48_row.txt"])
 def test_prepare_matches_hand_derived_row(name):
     g = load(name)
     x = (np.array(g["x_over_D"], dtype=np.float64) * g["D"]).astype(F32)[None, :]
