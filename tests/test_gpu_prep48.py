@@ -80,3 +80,19 @@ def test_prep48_not_executed_or_taken_elsewhere():
         with pytest.raises(S.SharqError) as e:
             call()
         assert e.value.status == S.SHARQ_ERR_UNSUPPORTED
+
+
+def test_prep48_hand_derived_row():
+    """The hand-derived MXFP4 4:8 row of tests/golden through the kernel (tiled to K=256)."""
+    from tests.golden_io import load
+    S = require_gpu()
+    g = load("mxfp4_elem48_row.txt")
+    row = (np.array(g["x_over_D"], dtype=np.float64) * g["D"]).astype(np.float32)
+    x_bits = wl.f32_to_bf16_bits(np.tile(row, 256 // row.size)[None, :].repeat(3, axis=0))
+    _, got, ref = prep48(S, x_bits, None, 1)
+    assert_exact(got, ref)
+    assert got["idx"][0, :8].reshape(-1).tolist() == g["idx"]
+    assert got["sp_codes"][0, :len(g["sp_codes"])].tolist() == g["sp_codes"]
+    assert got["res_codes"][0, :len(g["res_codes"])].tolist() == g["res_codes"]
+    assert got["sp_scales"][0, :1].tolist() == [g["sp_scales"]]
+    assert got["res_scales"][0, :2].tolist() == g["res_scales"]
