@@ -94,7 +94,7 @@ typedef enum { SHARQ_OUT_BF16 = 0, SHARQ_OUT_F32 = 1 } sharq_out;
 typedef enum {
   SHARQ_OK = 0,
   SHARQ_ERR_INVALID_ARG = 1, /* bad size, null pointer, misalignment, mismatched operands */
-  SHARQ_ERR_UNSUPPORTED = 2, /* valid request this build does not execute (e.g. a pattern) */
+  SHARQ_ERR_UNSUPPORTED = 2, /* valid request the library does not execute (e.g. a pattern) */
   SHARQ_ERR_CUDA = 3,        /* the CUDA runtime reported a launch or device error */
   SHARQ_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (see sharq_device_status) */
 } sharq_status;

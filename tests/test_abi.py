@@ -66,7 +66,7 @@ def test_wpack_buffer_sizes(S):
     ((16, 4096, 3, 2, 2, 0), 1),    # N > M
     ((16, 4096, 2, 4, 3, 0), 1),    # bad unit
     ((16, 4096, 2, 4, 2, 7), 1),    # bad format
-    ((16, 4096, 1, 4, 2, 0), 2),    # valid pattern this build does not compute
+    ((16, 4096, 1, 4, 2, 0), 2),    # valid pattern the library does not compute
     ((16, 4096, 4, 8, 2, 0), 2),    # 4:8 over pairs: not computed (4:8 is over elements)
 ])
 def test_prep_sizes_reject(S, args, status):
